@@ -1,0 +1,153 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) frozen-base NF4 LoRA linear layer.
+ *
+ * The layer is the QLoRA base linear: the frozen weight W0 [n_out, n_in] is
+ * stored as 4-bit NormalFloat codes in blocks of 64 with one absmax scale per
+ * block, and those scales are quantized again to 8 bits in groups of 256 with
+ * one fp32 constant per group ("QLoRA double quantization and block-wise
+ * quantization memory" page, sections 1.2, 2.2 and 2.3; "5.8 QLoRA: 4-bit
+ * base + 16-bit sticky notes" page, "three parts that make it work").  The
+ * forward pass is y = W0 x + (alpha / r) B (A x) ("Training LoRA directly on
+ * GGUF quantized weights" page, section 2.1 formula and section 3.2 module);
+ * the backward pass treats W0 as a read-only operator and returns dX, dA and
+ * dB (same page, section 2.1).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layouts are row-major.  W0 is [N, K] = [n_out, n_in]; X [M, K];
+ * A [r, K]; B [N, r]; Y [M, N]; dY [M, N]; dX [M, K]; U = X A^T [M, r];
+ * G = dY B [M, r].  bf16 tensors are passed as pointers to 16-bit words
+ * (qlora_bf16) holding IEEE bfloat16 bit patterns.
+ *
+ * Memory: every pointer is DEVICE memory owned by the caller, except where a
+ * parameter says "host".  The library allocates no device memory in any
+ * call; scratch space is the caller's `ws` buffer of at least
+ * qlora_workspace_bytes(...) bytes.  Device pointers must be 16-byte aligned.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  Calls only enqueue work; they do not synchronise.
+ *
+ * Errors: every call validates its arguments on the host before launching
+ * anything and returns a qlora_status; on failure nothing is launched and
+ * qlora_last_error() returns a message (thread-local).  Kernels never trap:
+ * a pipeline wait that exceeds its time limit (about two seconds) sets a
+ * device error word and the kernel returns; qlora_sync_status() reports it
+ * as QLORA_ERR_TIMEOUT.  Non-finite weights give unspecified codes.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t qlora_bf16;
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_ARG = 1,        /* null pointer, bad flag, bad scaling             */
+    QLORA_ERR_SHAPE = 2,      /* sizes out of range or not multiples of 64 / 8   */
+    QLORA_ERR_ALIGN = 3,      /* a device pointer is not 16-byte aligned         */
+    QLORA_ERR_WORKSPACE = 4,  /* ws missing or smaller than qlora_workspace_bytes */
+    QLORA_ERR_CUDA = 5,       /* a CUDA runtime call or launch failed            */
+    QLORA_ERR_TIMEOUT = 6,    /* a kernel gave up waiting (reported by sync)     */
+    QLORA_ERR_UNSUPPORTED = 7 /* no sm_100 device / wrong architecture           */
+} qlora_status;
+
+/* Packed NF4 + double-quant weight.  All three buffers are device memory
+ * owned by the caller.  numel = n_out * n_in must be a multiple of 64 and
+ * n_in must be a multiple of 64 (blocks never straddle rows).
+ *   codes   : numel / 2 bytes; weight element 2j (row-major flattening) is
+ *             in bits 0-3 of byte j, element 2j+1 in bits 4-7; each code
+ *             indexes the 16-entry NF4 codebook (see qlora_nf4_codebook).
+ *   scales  : numel / 64 bytes; block b (elements [64b, 64b+64)) has first
+ *             level scale q_b in 0..255.
+ *   scales2 : ceil(numel / 16384) floats; group g (blocks [256g, 256g+256))
+ *             has second-level step d_g.  The dequantized block scale is
+ *             s_b = fp32(q_b * d_g) and the weight is fp32(c[code] * s_b). */
+typedef struct {
+    int64_t n_out;
+    int64_t n_in;
+    uint8_t *codes;
+    uint8_t *scales;
+    float *scales2;
+} qlora_nf4_weight;
+
+/* Bytes of the three packed buffers together: numel/2 + numel/64 +
+ * 4*ceil(numel/16384) (the closed form of the "QLoRA double quantization"
+ * page, section 2.3).  Returns 0 if numel is not a positive multiple of 64. */
+size_t qlora_packed_bytes(int64_t numel);
+
+/* Writes the 16 NF4 levels (ascending float32, out[0] = -1, out[7] = 0,
+ * out[15] = +1) to the HOST array out.  The levels are the normal quantiles
+ * of the "5.8 QLoRA" page's NF4 paragraph: 8 positive and 7 negative
+ * quantiles at equal probability steps below the offset
+ * delta = ((1 - 1/30) + (1 - 1/32)) / 2, each divided by Phi^-1(delta),
+ * plus an exact zero.  Returns QLORA_ERR_ARG if out is NULL. */
+qlora_status qlora_nf4_codebook(float out[16]);
+
+/* Encode: W [n_out, n_in] fp32 (device) -> w->codes, w->scales, w->scales2.
+ * Per block of 64: a_b = max |w|; code = index of the nearest level to
+ * fp32(w / a_b), exact ties to the lower index (a_b = 0 gives code 7).
+ * Per group of 256 blocks: d_g = fp32(max a_b / 255) and
+ * q_b = clamp(round_half_even(fp32(a_b / d_g)), 0, 255) (d_g = 0 gives 0).
+ * Sections 1.2-2.3 of the "QLoRA double quantization" page.  Bit-exact. */
+qlora_status qlora_quantize_nf4_dq(const float *W, const qlora_nf4_weight *w, void *stream);
+
+/* Dequant the whole weight (the "one-shot dequant" route of the GGUF page,
+ * section 2.2): out [n_out, n_in] receives fp32(c[code] * fp32(q_b * d_g)),
+ * as float32 (out_is_bf16 = 0) or rounded to bfloat16 ties-to-even
+ * (out_is_bf16 = 1).  Bit-exact. */
+qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16, void *stream);
+
+/* Scratch bytes needed by qlora_lora_linear_fwd / qlora_lora_linear_bwd_dx for
+ * these sizes (N = n_out, K = n_in).  0 is never returned for valid sizes. */
+size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/* Forward: Y = X W'^T + scaling * (X A^T) B^T, W' the dequantized base.
+ *   X [M, K] bf16, A [r, K] bf16, B [N, r] bf16, Y [M, N] bf16 (output).
+ *   r = 0 disables the adapter (A, B may then be NULL); otherwise
+ *   8 <= r <= 128 and r % 8 == 0.  scaling = alpha / r, computed by the
+ *   caller (the GGUF page's section 3.2 module).
+ *   U_save [M, r] bf16 receives U = X A^T (needed by qlora_lora_grad_AB), or
+ *   NULL.  ws / ws_bytes: caller scratch of qlora_workspace_bytes(M, N, K, r).
+ * The base term is computed on tensor cores from bf16 operands with fp32
+ * accumulation; the weight operand is bf16(bf16(c[code]) * bf16(s_b)). */
+qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *X, int64_t M,
+                                   const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                   qlora_bf16 *Y, qlora_bf16 *U_save,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/* Backward to the input: dX = dY W' + scaling * (dY B) A  (the frozen base
+ * is a read-only operator; no gradient is formed for W0).
+ *   dY [M, N] bf16, dX [M, K] bf16 (output), G_save [M, r] bf16 receives
+ *   G = dY B, or NULL.  Other arguments as in qlora_lora_linear_fwd. */
+qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf16 *dY, int64_t M,
+                                      const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                      qlora_bf16 *dX, qlora_bf16 *G_save,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/* Adapter gradients ("only A and B are updated", course-notes page LoRA
+ * section): dA = scaling * G^T X  [r, K] fp32 and dB = scaling * dY^T U
+ * [N, r] fp32, with U and G as saved by the two calls above.  accumulate = 1
+ * adds into dA and dB, 0 overwrites them.  8 <= r <= 128, r % 8 == 0,
+ * K % 64 == 0, N % 64 == 0. */
+qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const qlora_bf16 *U,
+                                const qlora_bf16 *G, int64_t M, int64_t N, int64_t K, int r,
+                                float scaling, float *dA, float *dB, int accumulate, void *stream);
+
+/* Waits for `stream`, then reports and clears a device-side timeout
+ * recorded by any earlier kernel of this library on the current device. */
+qlora_status qlora_sync_status(void *stream);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char *qlora_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */
