@@ -8,8 +8,11 @@
 // into shared memory in the MN-major 128-byte-swizzled layout (k contiguous)
 // and the MMA reads A from there.  B (dY) arrives by TMA, K-major.
 //
-// Roles (384 threads): warp 0 dY/gs TMA producer, warp 1 MMA issuer, warp 2
-// TMEM allocator, warp 3 packed-code TMA producer, warps 4-11 dequant + epilogue.
+// Roles (640 threads): warp 0 TMA producer of the dY ring (read by the MMA only),
+// warp 3 TMA producer of the packed-code ring (slot s % 8 is read only by
+// dequant group s % 4, in stage order), warp 1 MMA issuer, warp 2 TMEM
+// allocator, warps 4-19 four dequant groups (group g takes stages s % 4 == g,
+// thread = one 64-block of a contraction row), then the epilogue.
 #pragma once
 
 #include <cstdint>
@@ -21,10 +24,11 @@ namespace qlora {
 namespace bwd {
 
 constexpr int BM = 128;                 // columns k of W0 per tile
-constexpr int SX = 4;                   // dY ring (64 n each)
-constexpr int SC = 4;                   // code ring (64 n x 128 k each)
-constexpr int SA = 2;                   // A ring in smem (W'^T tiles)
-constexpr int kDqWarps = 8;
+constexpr int SX = 3;                   // dY ring (64 n each)
+constexpr int SC = 8;                   // code ring (a multiple of kGroups)
+constexpr int kGroups = 4;              // dequant groups = smem A slots
+constexpr int SA = kGroups;             // A ring in smem (W'^T tiles)
+constexpr int kDqWarps = 4 * kGroups;
 constexpr int kThreads = 128 + 32 * kDqWarps;
 constexpr int kCodeStageBytes = 64 * 64;     // 64 rows x 64 bytes
 constexpr int kAStageBytes = 64 * 128 * 2;   // 64 n x 128 k bf16
@@ -41,9 +45,8 @@ struct Params {
     float level[16];
 };
 
-__host__ __device__ constexpr int y_stage_bytes(int BN) { return BN * 128; }
 __host__ __device__ constexpr int smem_bytes(int BN) {
-    return 1024 + SX * y_stage_bytes(BN) + SA * kAStageBytes + SC * kCodeStageBytes + kLutWords * 4 + 256;
+    return 1024 + SX * BN * 128 + SC * kCodeStageBytes + SA * kAStageBytes + kLutWords * 4 + 512 /*barriers*/;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) { return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u; }
 
@@ -52,7 +55,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmG, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int ysb = y_stage_bytes(p.BN);
+    const int ysb = p.BN * 128;
     uint8_t *sY = smem;
     uint8_t *sA = sY + SX * ysb;
     uint8_t *sC = sA + SA * kAStageBytes;
@@ -79,11 +82,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total = nmain + LS;
     const uint32_t ncols = tmem_cols(p.BN);
 
-    if (threadIdx.x < 16) s_level[threadIdx.x] = p.level[threadIdx.x];
+    if (threadIdx.x < 16) {
+        float v = 0.f;  // constant-index reads keep the parameter block out of local memory
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (threadIdx.x == i) v = p.level[i];
+        s_level[threadIdx.x] = v;
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; ++i) { mbar_init(&y_full[i], 1); mbar_init(&y_empty[i], 1); }
-        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], kDqWarps); }
-        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], kDqWarps); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 4); }
+        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -157,16 +166,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_drain(acc_full, 0);
         }
     } else if (warp >= 4) {
+        // thread = (contraction row nl, k half h): one 64-block of W0 row n
         const int dw = warp - 4;
-        const int nl = dw * 8 + (lane & 7);        // contraction row within the stage (0..63)
-        const int sub = lane >> 3;
-        const int h = sub >> 1, q = sub & 1;        // k half (64 k) and 32-k quarter inside it
+        const int grp = dw >> 2;                    // stages s with s % kGroups == grp
+        const int wi = dw & 3;
+        const int nl = (wi & 1) * 32 + lane;        // contraction row within the stage (0..63)
+        const int h = wi >> 1;                      // k half: columns k0 + 64h ..
         const int kblk = k0 / 64 + h;               // 64-block index along the row
         const bool kvalid = kblk < KB;
         const uint32_t lut = smem_u32(sLut) + lane * 4;
-        const uint32_t sCu = smem_u32(sC), sAu = smem_u32(sA);
-        const int cidx = h * 2 + q;
-        const uint32_t c_off = nl * 64 + ((cidx ^ ((nl >> 1) & 3)) << 4);
+        const uint32_t sAu = smem_u32(sA);
+        // 64-byte code rows, 64-byte swizzle: chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
+        const uint32_t c_row = smem_u32(sC) + nl * 64;
+        const uint32_t c_swz = (nl >> 1) & 3;
         const uint32_t a_off = h * 8192 + nl * 128;
         bool ok = true;
 
@@ -174,46 +186,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = (nb_begin + s) * 64 + nl;
             qv = 0;
             dv = 0.f;
-            if (kvalid && n < p.N) {
+            if (kvalid && s < nmain && n < p.N) {
                 const int64_t b = int64_t(n) * KB + kblk;
                 qv = __ldg(p.scales + b);
                 dv = __ldg(p.scales2 + (b >> 8));
             }
         };
-        uint32_t q_next;
-        float d_next;
-        load_scale(0, q_next, d_next);
+        // block scales of this group's next three stages (12 stages of lookahead)
+        uint32_t qa, qb, qc;
+        float da, db, dc;
+        load_scale(grp, qa, da);
+        load_scale(grp + kGroups, qb, db);
+        load_scale(grp + 2 * kGroups, qc, dc);
 
-        for (int s = 0; s < total && ok; ++s) {
-            const int sa = s % SA;
-            uint32_t out[16];
+        for (int s = grp; s < total && ok; s += kGroups) {
+            const int sc = s % SC, sa = s % SA;
+            uint32_t out[32];
             if (s < nmain) {
-                const int sc = s % SC;
                 if (!mbar_wait(&c_full[sc], (s / SC) & 1, abort_flag)) { ok = false; break; }
-                const float sv = __fmul_rn(static_cast<float>(q_next), d_next);
-                if (s + 1 < nmain) load_scale(s + 1, q_next, d_next);
+                const float sv = __fmul_rn(static_cast<float>(qa), da);
+                qa = qb; da = db; qb = qc; db = dc;
+                load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);
                 const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
-                const uint4 cw = lds128(sCu + sc * kCodeStageBytes + c_off);
+                const uint32_t cbase = c_row + sc * kCodeStageBytes;
+                const uint4 c0 = lds128(cbase + (((2u * h + 0u) ^ c_swz) << 4));
+                const uint4 c1 = lds128(cbase + (((2u * h + 1u) ^ c_swz) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c_empty[sc]);
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                for (int w4 = 0; w4 < 4; ++w4) {
+                for (int w8 = 0; w8 < 8; ++w8) {
 #pragma unroll
                     for (int by = 0; by < 4; ++by) {
-                        const uint32_t e = (words[w4] >> (8 * by)) & 0xFFu;
-                        out[w4 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                        const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
+                        out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
                     }
                 }
             } else {
-                // adapter chunk: rows j of A [r, K], 32 k starting at k0 + 64h + 32q (zero past r / K)
+                // adapter chunk: row j of A [r, K], 64 k starting at k0 + 64h (zero past r / K)
                 const int j = (s - nmain) * 64 + nl;
-                const int kk0 = k0 + h * 64 + q * 32;
+                const int kk0 = k0 + h * 64;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
+                for (int v = 0; v < 8; ++v) {
                     uint4 w = make_uint4(0, 0, 0, 0);
-                    if (j < p.r && kk0 + v * 8 < p.K)
+                    if (j < p.r && kk0 < p.K)
                         w = __ldg(reinterpret_cast<const uint4 *>(p.Alora + int64_t(j) * p.K + kk0 + v * 8));
                     out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
                 }
@@ -221,8 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&a_empty[sa], ((s / SA) & 1) ^ 1, abort_flag)) { ok = false; break; }
             const uint32_t abase = sAu + sa * kAStageBytes + a_off;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t chunk = (q * 4 + i) ^ (nl & 7);
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t chunk = uint32_t(i) ^ uint32_t(nl & 7);
                 sts128(abase + (chunk << 4), make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]));
             }
             fence_proxy_async_smem();
@@ -234,12 +251,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && mbar_wait(acc_full, 0, abort_flag)) {
             tc_fence_after();
             const int quad = warp & 3;
-            const int half = dw >> 2;
             const int row = quad * 32 + lane;
             const int k = k0 + row;
             const uint32_t lane_addr = uint32_t(quad * 32) << 16;
             const int nchunks = p.BN / 16;
-            for (int ch = half; ch < nchunks; ch += 2) {
+            for (int ch = grp; ch < nchunks; ch += kGroups) {
                 uint32_t v[16];
                 tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
                 tmem_wait_ld16(v);

@@ -5,16 +5,20 @@
 // with us = bf16(scaling * X A^T) prepared by a side kernel, so the adapter is
 // one or two extra K-chunks folded into the same TMEM accumulator.  Y = D^T.
 //
-// Roles (384 threads):
-//   warp 0      TMA producer for the X tile ring (and the us tiles of the adapter chunk)
-//   warp 1      MMA issuer (one thread): tcgen05.mma with A from TMEM, B (X) from smem
-//   warp 2      TMEM allocator
-//   warp 3      TMA producer for the packed-code ring
-//   warps 4-11  dequant: thread = one W row; 16 code bytes -> 32 bf16 via a
-//               byte->bf16x2 lookup table in shared memory, times the bf16 block
-//               scale, written straight into TMEM (the MMA's A operand);
-//               then the epilogue: TMEM -> registers -> bf16 Y (or fp32 atomics
-//               into a split-K accumulator).
+// Pipeline per 64-wide K stage s:
+//   producer (warp 0)   TMA load of the X tile [BN x 64] into the X ring (read by the MMA only)
+//   producer (warp 3)   TMA load of the packed codes for four stages [128 rows x 128 bytes]
+//                       into the code ring; every dequant group reads every chunk, in
+//                       chunk order, so no barrier is waited on two phases ahead
+//   dequant group s%4   (4 warps, thread = one W row, 64 weights) reads its row's 32
+//                       code bytes, expands each byte through a shared-memory table
+//                       byte -> (level[lo], level[hi]) as bf16x2, multiplies by the
+//                       bf16 block scale and stores the 32 columns into TMEM slot s%4
+//   MMA (warp 1)        four tcgen05.mma (K = 16) with A from TMEM, B (X) from smem
+// Four dequant groups work on four consecutive stages at once, so the TMEM
+// store and barrier latency of one stage overlaps the expansion of the next.
+// Epilogue: the dequant warps read the accumulator back (tcgen05.ld) and write
+// bf16 Y (or add fp32 partial sums into a split-K accumulator).
 #pragma once
 
 #include <cstdint>
@@ -26,12 +30,13 @@ namespace qlora {
 namespace fwd {
 
 constexpr int BM = 128;            // W rows per tile
-constexpr int SX = 4;              // X/us smem ring stages (64 K each)
-constexpr int SC = 2;              // code ring stages (256 K each)
-constexpr int SA = 4;              // TMEM A stages (64 K = 32 columns each)
-constexpr int kDqWarps = 8;
+constexpr int SX = 5;              // X ring stages (64 K each)
+constexpr int SC = 2;              // code ring chunks (256 K each, read by all four groups)
+constexpr int kGroups = 4;         // dequant groups = TMEM A slots (32 columns each)
+constexpr int SA = kGroups;
+constexpr int kDqWarps = 4 * kGroups;
 constexpr int kThreads = 128 + 32 * kDqWarps;
-constexpr int kCodeStageBytes = BM * 128;     // 128 rows x 128 bytes (256 weights)
+constexpr int kCodeChunkBytes = BM * 128;     // 128 rows x 128 bytes (256 weights = 4 stages)
 constexpr int kLutWords = 256 * 32;           // byte -> bf16x2, replicated per lane
 
 struct Params {
@@ -45,12 +50,11 @@ struct Params {
     float level[16];
 };
 
-__host__ __device__ constexpr int x_stage_bytes(int BN) { return BN * 128; }
 __host__ __device__ constexpr int smem_bytes(int BN) {
-    return 1024 /*align slack*/ + SX * x_stage_bytes(BN) + SC * kCodeStageBytes + kLutWords * 4 + 256;
+    return 1024 /*align slack*/ + SX * BN * 128 + SC * kCodeChunkBytes + kLutWords * 4 + 512 /*barriers*/;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
-    // A ring at columns [0, 128), accumulator at [128, 128 + BN)
+    // A slots at columns [0, 128), accumulator at [128, 128 + BN)
     return (128 + BN) <= 256 ? 256u : 512u;
 }
 
@@ -59,10 +63,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmU, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int xsb = x_stage_bytes(p.BN);
+    const int xsb = p.BN * 128;
     uint8_t *sX = smem;
     uint8_t *sC = sX + SX * xsb;
-    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeStageBytes);
+    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
     uint64_t *x_full = bars, *x_empty = bars + SX;
     uint64_t *c_full = bars + 2 * SX, *c_empty = c_full + SC;
@@ -84,11 +88,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total = nmain + LS;
     const uint32_t ncols = tmem_cols(p.BN);
 
-    if (threadIdx.x < 16) s_level[threadIdx.x] = p.level[threadIdx.x];
+    if (threadIdx.x < 16) {
+        float v = 0.f;  // constant-index reads keep the parameter block out of local memory
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (threadIdx.x == i) v = p.level[i];
+        s_level[threadIdx.x] = v;
+    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
         for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], kDqWarps); }
-        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], kDqWarps); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < SA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -108,11 +118,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_a = tmem;          // A stages: columns sa*32 .. sa*32+31
+    const uint32_t tmem_a = tmem;          // A slots: columns g*32 .. g*32+31
     const uint32_t tmem_acc = tmem + 128;  // accumulator: columns 128 .. 128+BN-1
 
     if (warp == 0) {
-        // ---------------- X / us producer
+        // ---------------- X producer (us tiles for the adapter chunks)
         if (lane == 0) {
             tma_prefetch_desc(&tmX);
             if (LS) tma_prefetch_desc(&tmU);
@@ -131,20 +141,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = max(0, issued - SX); s < issued; ++s) mbar_drain(&x_full[s % SX], (s / SX) & 1);
         }
     } else if (warp == 3) {
-        // ---------------- packed-code producer (256 weights per row per stage)
+        // ---------------- packed-code producer
         if (lane == 0) {
             tma_prefetch_desc(&tmC);
-            const int c_begin = kb_begin / 4;
-            const int c_end = (kb_end + 3) / 4;
+            // one 128-row x 128-byte tile (256 K, four stages) per chunk; kb_begin is a multiple of 4
+            const int nchunk = (nmain + 3) / 4;
             int issued = 0;
-            for (int c = c_begin; c < c_end; ++c) {
-                const int i = c - c_begin, sc = i % SC;
-                if (!mbar_wait(&c_empty[sc], ((i / SC) & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&c_full[sc], kCodeStageBytes);
-                tma_load_2d(sC + sc * kCodeStageBytes, &tmC, &c_full[sc], c * 128, n0);
-                issued = i + 1;
+            for (int c = 0; c < nchunk; ++c) {
+                const int sc = c % SC;
+                if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&c_full[sc], kCodeChunkBytes);
+                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], (kb_begin / 4 + c) * 128, n0);
+                issued = c + 1;
             }
-            for (int i = max(0, issued - SC); i < issued; ++i) mbar_drain(&c_full[i % SC], (i / SC) & 1);
+            for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer
@@ -171,63 +181,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= 4) {
         // ---------------- dequant into TMEM, then epilogue
         const int dw = warp - 4;
-        const int half = dw >> 2;                 // which 32 weights of each 64-block
+        const int grp = dw >> 2;                  // stages s with s % kGroups == grp
         const int quad = warp & 3;                // TMEM lane quadrant this warp may access
         const int row = quad * 32 + lane;         // W row within the tile
         const int n = n0 + row;
         const bool valid = n < p.N;
         const uint32_t lut = smem_u32(sLut) + lane * 4;
-        const uint32_t sCu = smem_u32(sC);
         const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        // 32-byte code row, 32-byte swizzle: chunk c of row r sits at chunk c ^ ((r >> 2) & 1)
+        const uint32_t code_row = smem_u32(sC) + row * 128;
+        const uint32_t cswz = row & 7;
         bool ok = true;
-        const int64_t row_block0 = int64_t(n) * KB;
-        // block scale of the next main stage, loaded one stage ahead
-        uint32_t q_next = 0;
-        float d_next = 0.f;
-        if (valid && nmain > 0) {
-            const int64_t b = row_block0 + kb_begin;
-            q_next = __ldg(p.scales + b);
-            d_next = __ldg(p.scales2 + (b >> 8));
-        }
+        const int64_t row_block0 = int64_t(n) * KB + kb_begin;
+        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
+            qv = 0;
+            dv = 0.f;
+            if (valid && s < nmain) {
+                const int64_t b = row_block0 + s;
+                qv = __ldg(p.scales + b);
+                dv = __ldg(p.scales2 + (b >> 8));
+            }
+        };
+        // block scales of this group's next three stages (12 stages of lookahead)
+        uint32_t qa, qb, qc;
+        float da, db, dc;
+        load_scale(grp, qa, da);
+        load_scale(grp + kGroups, qb, db);
+        load_scale(grp + 2 * kGroups, qc, dc);
 
-        for (int s = 0; s < total && ok; ++s) {
-            const int sa = s % SA;
-            uint32_t out[16];
+        for (int s = grp; s < total && ok; s += kGroups) {
+            const int ci = s >> 2, sc = ci % SC, sa = s % SA;
+            uint32_t out[32];
             if (s < nmain) {
-                const int kb = kb_begin + s;
-                const int ci = kb / 4 - kb_begin / 4;
-                const int sc = ci % SC;
-                if ((s == 0) || (kb % 4 == 0)) {
-                    if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
-                }
-                const float sv = __fmul_rn(static_cast<float>(q_next), d_next);
-                if (valid && s + 1 < nmain) {
-                    const int64_t b = row_block0 + kb + 1;
-                    q_next = __ldg(p.scales + b);
-                    d_next = __ldg(p.scales2 + (b >> 8));
-                }
+                if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
+                const float sv = __fmul_rn(static_cast<float>(qa), da);
+                qa = qb; da = db; qb = qc; db = dc;
+                load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);
                 const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
-                const int j = 2 * (kb & 3) + half;            // 16-byte chunk within the 128-byte row
-                const uint4 cw = lds128(sCu + sc * kCodeStageBytes + row * 128 + ((j ^ (row & 7)) << 4));
-                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                const uint32_t cbase = code_row + sc * kCodeChunkBytes;
+                const uint32_t j0 = 2u * uint32_t(s & 3);
+                const uint4 c0 = lds128(cbase + (((j0 + 0u) ^ cswz) << 4));
+                const uint4 c1 = lds128(cbase + (((j0 + 1u) ^ cswz) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                for (int w4 = 0; w4 < 4; ++w4) {
+                for (int w8 = 0; w8 < 8; ++w8) {
 #pragma unroll
                     for (int by = 0; by < 4; ++by) {
-                        const uint32_t e = (words[w4] >> (8 * by)) & 0xFFu;
-                        out[w4 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                        const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
+                        out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
                     }
                 }
-                if ((kb % 4 == 3) || (kb == kb_end - 1)) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&c_empty[sc]);
-                }
             } else {
-                // adapter chunk: A operand = B_lora row n, elements e0 .. e0+31 (zero past r)
-                const int e0 = (s - nmain) * 64 + half * 32;
+                // adapter chunk: A operand = B_lora row n, elements e0 .. e0+63 (zero past r)
+                const int e0 = (s - nmain) * 64;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
+                for (int v = 0; v < 8; ++v) {
                     uint4 q = make_uint4(0, 0, 0, 0);
                     if (valid && e0 + v * 8 < p.r)
                         q = __ldg(reinterpret_cast<const uint4 *>(p.Blora + int64_t(n) * p.r + e0 + v * 8));
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!mbar_wait(&a_empty[sa], ((s / SA) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            tmem_st16(tmem_a + lane_addr + sa * 32 + half * 16, out);
+            tmem_st32(tmem_a + lane_addr + sa * 32, out);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && mbar_wait(acc_full, 0, abort_flag)) {
             tc_fence_after();
             const int nchunks = p.BN / 16;
-            for (int ch = half; ch < nchunks; ch += 2) {
+            for (int ch = grp; ch < nchunks; ch += kGroups) {
                 uint32_t v[16];
                 tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
                 tmem_wait_ld16(v);

@@ -1,0 +1,311 @@
+// fused_fwd_pair.cuh -- forward GEMM with NF4 dequant, on CTA pairs (tcgen05 cta_group::2).
+//
+//   D[n, m] = sum_k W'[n, k] X[m, k] (+ adapter chunk),  n in 256 rows (128 per CTA), m in BN tokens
+//
+// Two CTAs on two SMs form one 256-row x BN-token tile.  Each CTA dequantizes
+// its own 128 W rows into its own TMEM (the MMA's A operand) and loads only its
+// half of the token tile (BN/2 rows of X) into its own shared memory; one
+// tcgen05.mma.cta_group::2 issued by the even CTA reads both halves.
+//
+// The MMA issue is effectively synchronous with the issuing thread, so every
+// barrier operation of that thread is lost tensor time.  The pipeline is built
+// to keep them rare: a stage is 128 K (eight MMAs) with one full-barrier wait
+// for X, one for the dequantized A slot, and one commit for each.
+//   producer (warp 0)    one 3-D TMA instruction per stage: two 64-K chunks of
+//                        this CTA's X half, counted on the even CTA's x_full
+//   producer (warp 3)    packed codes, 256 K (two stages) per TMA instruction
+//   dequant group q % 4  (4 warps, thread = one W row) expands the stage's 128
+//                        weights of its row through a shared-memory table
+//                        byte -> (level[lo], level[hi]) as bf16x2 times the bf16
+//                        block scale, into TMEM slot q % 4 (64 columns), then
+//                        arrives on the even CTA's a_full
+//   MMA (warp 1, even)   eight tcgen05.mma (K = 16), A from TMEM, B from smem
+// Commits are multicast to both CTAs (x_empty, a_empty, acc_full).  Each CTA
+// finally reads back its own 128 x BN accumulator.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace qlora {
+namespace fwdp {
+
+constexpr int BM = 128;            // W rows per CTA (256 per pair)
+constexpr int kStageK = 128;       // K per pipeline stage (two 64-K chunks, eight MMAs)
+constexpr int SX = 3;              // X ring slots (one stage each)
+constexpr int SC = 4;              // code ring chunks (256 K = two stages each)
+constexpr int kGroups = 4;         // dequant groups = TMEM A slots (64 columns each)
+constexpr int kDqWarps = 4 * kGroups;
+constexpr int kThreads = 128 + 32 * kDqWarps;
+constexpr int kCodeChunkBytes = BM * 128;     // 128 rows x 128 bytes (256 weights)
+constexpr int kLutWords = 256 * 32;           // byte -> bf16x2, replicated per lane
+
+struct Params {
+    const uint8_t *scales;
+    const float *scales2;
+    const uint16_t *Blora;   // [N, r] bf16 or nullptr
+    uint16_t *Y;             // [M, N] bf16
+    int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
+    float level[16];
+};
+
+__host__ __device__ constexpr int smem_bytes(int BN) {
+    return 1024 /*align slack*/ + SX * 2 * (BN / 2) * 128 + SC * kCodeChunkBytes + kLutWords * 4 + 512 /*barriers*/;
+}
+// A slots at columns [0, 256), accumulator at [256, 256 + BN)
+__host__ __device__ constexpr uint32_t tmem_cols(int) { return 512u; }
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    fused_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
+                          const __grid_constant__ CUtensorMap tmU, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int half_bn = p.BN / 2;
+    const int xsb = half_bn * 128;               // this CTA's half X tile for one 64-K chunk
+    const int slotb = 2 * xsb;                   // one X ring slot (one stage)
+    uint8_t *sX = smem;
+    uint8_t *sC = sX + SX * slotb;
+    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
+    uint64_t *x_full = bars, *x_empty = bars + SX;
+    uint64_t *c_full = bars + 2 * SX, *c_empty = c_full + SC;
+    uint64_t *a_full = c_empty + SC, *a_empty = a_full + kGroups;
+    uint64_t *acc_full = a_empty + kGroups;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *s_level = reinterpret_cast<float *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();      // 0: even CTA (issues the MMAs), 1: its peer
+    const int n0 = blockIdx.x * BM;               // blockIdx.x = 2 * pair + rank
+    const int m0 = blockIdx.y * p.BN;
+    const int my_m0 = m0 + int(rank) * half_bn;
+    const int KB = p.K / 64;                      // 64-K chunks of the base
+    const int QM = (KB + 1) / 2;                  // main stages
+    const int Q = QM + (p.r > 0 ? 1 : 0);         // + one adapter stage (r <= 128)
+    const int nchunk = (KB + 3) / 4;              // 256-K code chunks
+
+    if (threadIdx.x < 16) {
+        float v = 0.f;  // constant-index reads keep the parameter block out of local memory
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (threadIdx.x == i) v = p.level[i];
+        s_level[threadIdx.x] = v;
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+        // a chunk is read by the two groups of its two stages
+        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 8); }
+        for (int i = 0; i < kGroups; ++i) { mbar_init(&a_full[i], 8); mbar_init(&a_empty[i], 1); }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(tmem_slot, tmem_cols(p.BN));
+        tmem_relinquish_pair();
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
+        const int e = i >> 5;
+        __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
+        sLut[i] = *reinterpret_cast<uint32_t *>(&v);
+    }
+    tc_fence_before();
+    // both CTAs' barriers are initialised before either signals the other's
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_a = tmem;          // A slots: columns g*64 .. g*64+63
+    const uint32_t tmem_acc = tmem + 256;  // accumulator: columns 256 .. 256+BN-1
+
+    if (warp == 0) {
+        // ---------------- X producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmX);
+            if (p.r > 0) tma_prefetch_desc(&tmU);
+            int issued = 0;
+            for (int q = 0; q < Q; ++q) {
+                const int sx = q % SX;
+                if (!mbar_wait(&x_empty[sx], ((q / SX) & 1) ^ 1, abort_flag)) break;
+                const uint32_t bar0 = mapa_shared(smem_u32(&x_full[sx]), 0);
+                uint8_t *slot = sX + sx * slotb;
+                if (q < QM) {
+                    if (rank == 0) mbar_arrive_expect_tx(&x_full[sx], 2 * slotb);
+                    tma_load_3d_pair(slot, &tmX, bar0, 0, my_m0, 2 * q);
+                } else {
+                    const int nv = (p.r + 63) / 64;
+                    if (rank == 0) mbar_arrive_expect_tx(&x_full[sx], 2 * nv * xsb);
+                    for (int d = 0; d < nv; ++d) tma_load_2d_pair(slot + d * xsb, &tmU, bar0, d * 64, my_m0);
+                }
+                issued = q + 1;
+            }
+            // the even CTA sees both CTAs' copies complete on its barriers
+            if (rank == 0)
+                for (int q = max(0, issued - SX); q < issued; ++q) mbar_drain(&x_full[q % SX], (q / SX) & 1);
+        }
+    } else if (warp == 3) {
+        // ---------------- packed-code producer (local to each CTA)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmC);
+            int issued = 0;
+            for (int c = 0; c < nchunk; ++c) {
+                const int sc = c % SC;
+                if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&c_full[sc], kCodeChunkBytes);
+                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], c * 128, n0);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (even CTA only)
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = make_idesc_bf16(2 * BM, p.BN, 0, 0);
+            for (int q = 0; q < Q; ++q) {
+                const int sx = q % SX, g = q % kGroups;
+                if (!mbar_wait(&x_full[sx], (q / SX) & 1, abort_flag)) break;
+                if (!mbar_wait(&a_full[g], (q / kGroups) & 1, abort_flag)) break;
+                tc_fence_after();
+                // MMAs of this stage: 8 for a full main stage, 4 for the last odd chunk,
+                // ceil(r/16) for the adapter stage
+                const int nk = q < QM ? (2 * q + 1 < KB ? 8 : 4) : (p.r + 15) / 16;
+                const uint32_t xbase = smem_u32(sX + sx * slotb);
+                for (int kk = 0; kk < nk; ++kk) {
+                    const uint64_t bdesc = make_sdesc_sw128(xbase + (kk >> 2) * xsb + (kk & 3) * 32, 16, 1024);
+                    mma_ts_pair(tmem_acc, tmem_a + g * 64 + kk * 8, bdesc, idesc, (q > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit_pair(&a_empty[g]);
+                tc_commit_pair(&x_empty[sx]);
+            }
+            tc_commit_pair(acc_full);
+            mbar_drain(acc_full, 0);
+        }
+    } else if (warp >= 4) {
+        // ---------------- dequant into this CTA's TMEM, then epilogue
+        const int dw = warp - 4;
+        const int grp = dw >> 2;
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int n = n0 + row;
+        const bool valid = n < p.N;
+        const uint32_t lut = smem_u32(sLut) + lane * 4;
+        const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        // 128-byte code rows, 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r & 7)
+        const uint32_t code_row = smem_u32(sC) + row * 128;
+        const uint32_t cswz = row & 7;
+        bool ok = true;
+        const int64_t row_block0 = int64_t(n) * KB;
+        auto load_scale = [&](int kb, uint32_t &qv, float &dv) {
+            qv = 0;
+            dv = 0.f;
+            if (valid && kb < KB) {
+                const int64_t b = row_block0 + kb;
+                qv = __ldg(p.scales + b);
+                dv = __ldg(p.scales2 + (b >> 8));
+            }
+        };
+        // block scales of this group's current and next stage (two 64-blocks each)
+        uint32_t qa0, qa1, qb0, qb1;
+        float da0, da1, db0, db1;
+        load_scale(2 * grp, qa0, da0);
+        load_scale(2 * grp + 1, qa1, da1);
+        load_scale(2 * (grp + kGroups), qb0, db0);
+        load_scale(2 * (grp + kGroups) + 1, qb1, db1);
+
+        for (int q = grp; q < Q && ok; q += kGroups) {
+            const int g = grp;
+            if (!mbar_wait(&a_empty[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (q < QM) {
+                const int ci = q >> 1, sc = ci % SC;
+                if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
+                const uint32_t cbase = code_row + sc * kCodeChunkBytes;
+                const uint32_t jq = 4u * uint32_t(q & 1);          // first 16-byte chunk of this stage
+                const uint4 c0 = lds128(cbase + (((jq + 0u) ^ cswz) << 4));
+                const uint4 c1 = lds128(cbase + (((jq + 1u) ^ cswz) << 4));
+                const uint4 c2 = lds128(cbase + (((jq + 2u) ^ cswz) << 4));
+                const uint4 c3 = lds128(cbase + (((jq + 3u) ^ cswz) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+                const float sv0 = __fmul_rn(static_cast<float>(qa0), da0);
+                const float sv1 = __fmul_rn(static_cast<float>(qa1), da1);
+                qa0 = qb0; da0 = db0; qa1 = qb1; da1 = db1;
+                load_scale(2 * (q + 2 * kGroups), qb0, db0);
+                load_scale(2 * (q + 2 * kGroups) + 1, qb1, db1);
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (sub == 1 && 2 * q + 1 >= KB) break;   // odd last chunk
+                    __nv_bfloat162 s2b = __float2bfloat162_rn(sub ? sv1 : sv0);
+                    const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
+                    const uint4 ca = sub ? c2 : c0, cb = sub ? c3 : c1;
+                    const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                    uint32_t out[32];
+#pragma unroll
+                    for (int w8 = 0; w8 < 8; ++w8) {
+#pragma unroll
+                        for (int by = 0; by < 4; ++by) {
+                            const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
+                            out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                        }
+                    }
+                    tmem_st32(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                }
+            } else {
+                // adapter stage: A operand = B_lora row n, elements 0 .. 127 (zero past r)
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (sub * 64 >= p.r) break;
+                    uint32_t out[32];
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        uint4 w = make_uint4(0, 0, 0, 0);
+                        const int e0 = sub * 64 + v * 8;
+                        if (valid && e0 < p.r)
+                            w = __ldg(reinterpret_cast<const uint4 *>(p.Blora + int64_t(n) * p.r + e0));
+                        out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
+                    }
+                    tmem_st32(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
+        }
+
+        // ---------------- epilogue: this CTA's 128 rows x BN tokens
+        if (ok && mbar_wait(acc_full, 0, abort_flag)) {
+            tc_fence_after();
+            const int nchunks = p.BN / 16;
+            for (int ch = grp; ch < nchunks; ch += kGroups) {
+                uint32_t v[16];
+                tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
+                tmem_wait_ld16(v);
+                if (valid) {
+                    const int mb = m0 + ch * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (mb + i < p.M) {
+                            __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+                            p.Y[int64_t(mb + i) * p.N + n] = *reinterpret_cast<uint16_t *>(&h);
+                        }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // neither CTA leaves (or frees TMEM) while the pair may still touch its memory
+    cluster_sync();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, tmem_cols(p.BN));
+    }
+}
+
+}  // namespace fwdp
+}  // namespace qlora

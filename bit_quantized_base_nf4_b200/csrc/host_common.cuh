@@ -12,7 +12,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
-#include "../../include/qlora_nf4.h"
+#include "qlora_nf4.h"
 
 namespace qlora {
 
@@ -144,6 +144,26 @@ static qlora_status make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMap
     if (r != CUDA_SUCCESS)
         return fail(QLORA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rows=%llu cols=%llu box=%ux%u", int(r),
                     (unsigned long long)rows, (unsigned long long)cols, box_rows, box_cols);
+    return QLORA_OK;
+}
+
+// 3-D map viewing a row-major [rows, cols] bf16 tensor as [cols/64 chunks][rows][64]:
+// one box = `depth` consecutive 64-column chunks of `box_rows` rows, each chunk a
+// 128-byte-swizzled [box_rows x 128 B] tile, stored chunk after chunk.
+static qlora_status make_tmap_chunks(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                                     uint32_t box_rows, uint32_t depth) {
+    auto fn = encode_fn();
+    if (!fn) return fail(QLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    cuuint64_t dims[3] = {64, rows, (cols + 63) / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, depth};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QLORA_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d) rows=%llu cols=%llu box=%ux64x%u", int(r),
+                    (unsigned long long)rows, (unsigned long long)cols, box_rows, depth);
     return QLORA_OK;
 }
 

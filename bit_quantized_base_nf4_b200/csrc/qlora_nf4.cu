@@ -7,8 +7,9 @@
 #include "host_common.cuh"
 #include "ptx.cuh"
 #include "quant_kernels.cuh"
-#include "lora_kernels.cuh"
+#include "skinny_mma.cuh"
 #include "fused_fwd.cuh"
+#include "fused_fwd_pair.cuh"
 #include "fused_bwd.cuh"
 
 using namespace qlora;
@@ -59,22 +60,81 @@ GemmPlan plan_gemm(int64_t M, int64_t rows, int64_t stages) {
         const int64_t maxs = std::max<int64_t>(1, stages / 4);
         splits = static_cast<int>(std::min(want, maxs));
     }
-    g.stages_per_split = static_cast<int>(ceil_div(stages, splits));
+    // whole four-stage code chunks per split
+    g.stages_per_split = static_cast<int>(ceil_div(ceil_div(stages, splits), 4) * 4);
     g.splits = static_cast<int>(ceil_div(stages, g.stages_per_split));
     return g;
 }
 
+template <typename K>
+qlora_status set_smem(K kernel, int bytes) {
+    return cuda_check(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                      "cudaFuncSetAttribute(max dynamic smem)");
+}
+
+qlora_status launch_check(const char *what) { return cuda_check(cudaGetLastError(), what); }
+
+// Workspace layout of the forward / dX calls:
+//   [0, a)      bf16 [M, r]   scaling * (X A^T) or scaling * (dY B): the adapter chunk operand
+//   [a, a+b)    fp32 [M, r]   accumulator of that rank-r product
+//   [a+b, ...)  fp32 [M, N] or [M, K]  split-K accumulator (small-M shapes only)
+struct WsLayout {
+    size_t rank_bf16, rank_acc, split_acc, total;
+};
+WsLayout ws_layout(int64_t M, int64_t rows, int r, bool split) {
+    WsLayout w;
+    w.rank_bf16 = round256(size_t(M) * size_t(std::max(r, 0)) * 2);
+    w.rank_acc = round256(size_t(M) * size_t(std::max(r, 0)) * 4);
+    w.split_acc = split ? round256(size_t(M) * size_t(rows) * 4) : 0;
+    w.total = w.rank_bf16 + w.rank_acc + w.split_acc;
+    return w;
+}
+// Forward kernel choice: CTA pairs (cta_group::2, 256 W rows per tile) from 64
+// tokens up; the single-CTA kernel with split-K below that (decode shapes).
+bool use_pair_fwd(int64_t M) { return M >= 64; }
+int pair_token_tile(int64_t M) {
+    const int64_t tiles = ceil_div(M, 256);
+    const int64_t bn = ceil_div(ceil_div(M, tiles), 32) * 32;
+    return static_cast<int>(std::max<int64_t>(32, std::min<int64_t>(256, bn)));
+}
 size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    const GemmPlan g = plan_gemm(M, N, K / 64);
-    size_t b = round256(size_t(M) * size_t(std::max(r, 0)) * 2);
-    if (g.splits > 1) b += round256(size_t(M) * size_t(N) * 4);
-    return b;
+    const bool split = !use_pair_fwd(M) && plan_gemm(M, N, K / 64).splits > 1;
+    return ws_layout(M, N, r, split).total;
 }
 size_t bwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    const GemmPlan g = plan_gemm(M, K, ceil_div(N, 64));
-    size_t b = round256(size_t(M) * size_t(std::max(r, 0)) * 2);
-    if (g.splits > 1) b += round256(size_t(M) * size_t(K) * 4);
-    return b;
+    return ws_layout(M, K, r, plan_gemm(M, K, ceil_div(N, 64)).splits > 1).total;
+}
+
+// Launches the rank-r tensor-core product (see skinny_mma.cuh); the output must
+// already hold zeros or the values to accumulate into.
+qlora_status launch_skinny(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_mn, int b_mn, int64_t T, int64_t I,
+                           int r, float scaling, float *out, int64_t ld_row, int64_t ld_col, cudaStream_t st) {
+    const int64_t ST = ceil_div(T, 64);
+    const int64_t tiles = ceil_div(I, skinny::BI);
+    const int64_t want = std::max<int64_t>(1, ceil_div(2 * sm_count(), tiles));
+    const int64_t sps = ceil_div(ST, std::min(ST, want));
+    skinny::Params p;
+    p.T = static_cast<int>(T);
+    p.I = static_cast<int>(I);
+    p.r = r;
+    p.stages_per_split = static_cast<int>(sps);
+    p.a_mn = a_mn;
+    p.b_mn = b_mn;
+    p.scaling = scaling;
+    p.out = out;
+    p.ld_row = ld_row;
+    p.ld_col = ld_col;
+    QL_TRY(set_smem(skinny::skinny_mma_kernel, skinny::smem_bytes()));
+    dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(ceil_div(ST, sps)));
+    skinny::skinny_mma_kernel<<<grid, skinny::kThreads, skinny::smem_bytes(), st>>>(tmA, tmB, p);
+    return launch_check("skinny_mma_kernel launch");
+}
+
+qlora_status launch_finalize(const float *acc, int64_t n, float scaling, uint16_t *save, uint16_t *scaled,
+                             cudaStream_t st) {
+    skinny::finalize_rank_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 2048)), 256, 0, st>>>(
+        acc, n, scaling, save, scaled);
+    return launch_check("finalize_rank_kernel launch");
 }
 
 qlora_status check_rank(int r, float scaling, const void *A, const void *B) {
@@ -94,13 +154,6 @@ qlora_status check_ws(void *ws, size_t ws_bytes, size_t need) {
     return QLORA_OK;
 }
 
-template <typename K>
-qlora_status set_smem(K kernel, int bytes) {
-    return cuda_check(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
-                      "cudaFuncSetAttribute(max dynamic smem)");
-}
-
-qlora_status launch_check(const char *what) { return cuda_check(cudaGetLastError(), what); }
 
 }  // namespace
 
@@ -185,17 +238,54 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
+    const bool pair = use_pair_fwd(M);
     const GemmPlan g = plan_gemm(M, N, K / 64);
-    uint16_t *us = static_cast<uint16_t *>(ws);
-    float *yacc = g.splits > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + round256(size_t(M) * r * 2))
-                               : nullptr;
+    const bool split = !pair && g.splits > 1;
+    const WsLayout L = ws_layout(M, N, r, split);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint16_t *us = reinterpret_cast<uint16_t *>(wsb);
+    float *uacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
+    float *yacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
     if (r > 0) {
-        lora_proj_kernel<<<static_cast<unsigned>(ceil_div(M, kProjTM)), 256, 0, st>>>(X, M, K, A, K, 1, r, scaling,
-                                                                                       U_save, us);
-        QL_TRY(launch_check("lora_proj_kernel (X A^T) launch"));
+        // U^T = A . X^T on tensor cores, then bf16 copies: U (saved) and scaling * U (adapter chunk)
+        CUtensorMap tA, tB;
+        QL_TRY(make_tmap_2d(&tA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, K, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(make_tmap_2d(&tB, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, 256, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(cuda_check(cudaMemsetAsync(uacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
+        QL_TRY(launch_skinny(tA, tB, 0, 0, K, M, r, 1.0f, uacc, 1, r, st));
+        QL_TRY(launch_finalize(uacc, M * r, scaling, U_save, us, st));
     }
-    if (yacc) QL_TRY(cuda_check(cudaMemsetAsync(yacc, 0, size_t(M) * N * 4, st), "zero split accumulator"));
+    const Codebook &cb = codebook();
 
+    if (pair) {
+        const int BN = pair_token_tile(M);
+        CUtensorMap tmX, tmC, tmU;
+        QL_TRY(make_tmap_chunks(&tmX, X, M, K, BN / 2, 2));
+        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+        if (r > 0)
+            QL_TRY(make_tmap_2d(&tmU, us, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
+                                CU_TENSOR_MAP_SWIZZLE_128B));
+        else
+            tmU = tmX;
+        fwdp::Params p;
+        p.scales = w->scales;
+        p.scales2 = w->scales2;
+        p.Blora = B;
+        p.Y = Y;
+        p.M = static_cast<int>(M);
+        p.N = static_cast<int>(N);
+        p.K = static_cast<int>(K);
+        p.r = r;
+        p.BN = BN;
+        for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
+        QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel, fwdp::smem_bytes(256)));
+        dim3 grid(static_cast<unsigned>(2 * ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, BN)), 1);
+        fwdp::fused_fwd_pair_kernel<<<grid, fwdp::kThreads, fwdp::smem_bytes(BN), st>>>(tmX, tmC, tmU, p);
+        return launch_check("fused_fwd_pair_kernel launch");
+    }
+
+    if (yacc) QL_TRY(cuda_check(cudaMemsetAsync(yacc, 0, size_t(M) * N * 4, st), "zero split accumulator"));
     CUtensorMap tmX, tmC, tmU;
     QL_TRY(make_tmap_2d(&tmX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, g.BN, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
@@ -219,7 +309,6 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     p.r = r;
     p.BN = g.BN;
     p.kb_per_split = g.stages_per_split;
-    const Codebook &cb = codebook();
     for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
 
     const int smem = fwd::smem_bytes(g.BN);
@@ -227,11 +316,7 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     dim3 grid(static_cast<unsigned>(g.tiles_rows), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
     fwd::fused_fwd_kernel<<<grid, fwd::kThreads, smem, st>>>(tmX, tmC, tmU, p);
     QL_TRY(launch_check("fused_fwd_kernel launch"));
-    if (yacc) {
-        const int64_t n = M * N;
-        f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 4096)), 256, 0, st>>>(yacc, Y, n);
-        QL_TRY(launch_check("split finalize launch"));
-    }
+    if (yacc) QL_TRY(launch_finalize(yacc, M * N, 1.0f, Y, nullptr, st));
     return QLORA_OK;
 }
 
@@ -252,13 +337,19 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     const GemmPlan g = plan_gemm(M, K, ceil_div(N, 64));
-    uint16_t *gs = static_cast<uint16_t *>(ws);
-    float *dxacc = g.splits > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + round256(size_t(M) * r * 2))
-                                : nullptr;
+    const WsLayout L = ws_layout(M, K, r, g.splits > 1);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint16_t *gs = reinterpret_cast<uint16_t *>(wsb);
+    float *gacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
+    float *dxacc = g.splits > 1 ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
     if (r > 0) {
-        lora_proj_kernel<<<static_cast<unsigned>(ceil_div(M, kProjTM)), 256, 0, st>>>(dY, M, N, B, 1, r, r, scaling,
-                                                                                       G_save, gs);
-        QL_TRY(launch_check("lora_proj_kernel (dY B) launch"));
+        // G^T = B^T . dY^T on tensor cores (B read MN-major), then bf16 copies G and scaling * G
+        CUtensorMap tA, tB;
+        QL_TRY(make_tmap_2d(&tA, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(make_tmap_2d(&tB, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, 256, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(cuda_check(cudaMemsetAsync(gacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
+        QL_TRY(launch_skinny(tA, tB, 1, 0, N, M, r, 1.0f, gacc, 1, r, st));
+        QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
     }
     if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
 
@@ -294,10 +385,7 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     bwd::fused_bwd_dx_kernel<<<grid, bwd::kThreads, smem, st>>>(tmY, tmC, tmG, p);
     QL_TRY(launch_check("fused_bwd_dx_kernel launch"));
     if (dxacc) {
-        const int64_t n = M * K;
-        f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 4096)), 256, 0, st>>>(dxacc, dX,
-                                                                                                            n);
-        QL_TRY(launch_check("split finalize launch"));
+        QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
     }
     return QLORA_OK;
 }
@@ -311,6 +399,7 @@ qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const
     if (M <= 0 || N <= 0 || K <= 0 || M > INT32_MAX || N > INT32_MAX || K > INT32_MAX)
         return fail(QLORA_ERR_SHAPE, "M, N and K must be in [1, 2^31)");
     if (r < 8 || r > 128 || r % 8) return fail(QLORA_ERR_SHAPE, "r (%d) must be a multiple of 8 in [8, 128]", r);
+    if (K % 64 || N % 8) return fail(QLORA_ERR_SHAPE, "K must be a multiple of 64 and N a multiple of 8");
     if (accumulate != 0 && accumulate != 1) return fail(QLORA_ERR_ARG, "accumulate must be 0 or 1");
     if (!std::isfinite(scaling)) return fail(QLORA_ERR_ARG, "scaling must be finite");
     QL_TRY(require_sm100());
@@ -319,13 +408,14 @@ qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const
         QL_TRY(cuda_check(cudaMemsetAsync(dA, 0, size_t(r) * K * 4, st), "zero dA"));
         QL_TRY(cuda_check(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st), "zero dB"));
     }
-    const unsigned ms = static_cast<unsigned>(ceil_div(M, kGradMPerCta));
-    lora_grad_kernel<<<dim3(static_cast<unsigned>(ceil_div(K, kGradTI)), ms), 256, 0, st>>>(X, M, K, G, r, scaling, dA,
-                                                                                           1, K);
-    QL_TRY(launch_check("lora_grad_kernel (dA) launch"));
-    lora_grad_kernel<<<dim3(static_cast<unsigned>(ceil_div(N, kGradTI)), ms), 256, 0, st>>>(dY, M, N, U, r, scaling, dB,
-                                                                                           r, 1);
-    QL_TRY(launch_check("lora_grad_kernel (dB) launch"));
+    // dA [r, K] = s G^T X  and  dB^T [r, N] = s U^T dY, contraction over the M tokens
+    CUtensorMap tG, tX, tU, tY;
+    QL_TRY(make_tmap_2d(&tG, G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    QL_TRY(make_tmap_2d(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    QL_TRY(make_tmap_2d(&tU, U, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    QL_TRY(make_tmap_2d(&tY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+    QL_TRY(launch_skinny(tG, tX, 1, 1, M, K, r, scaling, dA, K, 1, st));
+    QL_TRY(launch_skinny(tU, tY, 1, 1, M, N, r, scaling, dB, 1, r, st));
     return QLORA_OK;
 }
 

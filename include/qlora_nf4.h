@@ -134,7 +134,7 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
  * section): dA = scaling * G^T X  [r, K] fp32 and dB = scaling * dY^T U
  * [N, r] fp32, with U and G as saved by the two calls above.  accumulate = 1
  * adds into dA and dB, 0 overwrites them.  8 <= r <= 128, r % 8 == 0,
- * K % 64 == 0, N % 64 == 0. */
+ * K % 64 == 0, N % 8 == 0. */
 qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const qlora_bf16 *U,
                                 const qlora_bf16 *G, int64_t M, int64_t N, int64_t K, int r,
                                 float scaling, float *dA, float *dB, int accumulate, void *stream);

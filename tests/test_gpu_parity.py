@@ -230,5 +230,7 @@ def test_grad_accumulate_adds():
     dA2, dB2 = r.dA.clone(), r.dB.clone()
     q.qlora_lora_grad_AB(r.X, r.dY, r.U, r.G, c.r, c.scaling, dA2, dB2, accumulate=True)
     q.qlora_sync_status()
-    torch.testing.assert_close(dA2, 2 * r.dA, rtol=1e-5, atol=1e-7)
-    torch.testing.assert_close(dB2, 2 * r.dB, rtol=1e-5, atol=1e-7)
+    # partial sums are added with float atomics, so the order (and the last bits) may differ
+    for got, one in ((dA2, r.dA), (dB2, r.dB)):
+        scale = float(one.abs().max())
+        torch.testing.assert_close(got, 2 * one, rtol=1e-4, atol=1e-5 * scale)
