@@ -9,8 +9,10 @@
 //
 // The MMA issue is effectively synchronous with the issuing thread, so every
 // barrier operation of that thread is lost tensor time.  The pipeline is built
-// to keep them rare: a stage is 128 K (eight MMAs) with one full-barrier wait
-// for X, one for the dequantized A slot, and one commit for each.
+// to keep them rare: a stage is 128 K (eight MMAs), the MMA thread waits on one
+// barrier per stage (a_full, which the even CTA's dequant warps only arrive on
+// after they have seen the stage's X tile land) and commits once per stage to
+// free[s % 4], which releases both the X slot and the TMEM A slot of the stage.
 //   producer (warp 0)    one 3-D TMA instruction per stage: two 64-K chunks of
 //                        this CTA's X half, counted on the even CTA's x_full
 //   producer (warp 3)    packed codes, 256 K (two stages) per TMA instruction
@@ -20,7 +22,7 @@
 //                        block scale, into TMEM slot q % 4 (64 columns), then
 //                        arrives on the even CTA's a_full
 //   MMA (warp 1, even)   eight tcgen05.mma (K = 16), A from TMEM, B from smem
-// Commits are multicast to both CTAs (x_empty, a_empty, acc_full).  Each CTA
+// Commits are multicast to both CTAs (free, acc_full).  Each CTA
 // finally reads back its own 128 x BN accumulator.
 #pragma once
 
@@ -34,7 +36,7 @@ namespace fwdp {
 
 constexpr int BM = 128;            // W rows per CTA (256 per pair)
 constexpr int kStageK = 128;       // K per pipeline stage (two 64-K chunks, eight MMAs)
-constexpr int SX = 3;              // X ring slots (one stage each)
+constexpr int SX = 4;              // X ring slots (one stage each) = dequant groups
 constexpr int SC = 4;              // code ring chunks (256 K = two stages each)
 constexpr int kGroups = 4;         // dequant groups = TMEM A slots (64 columns each)
 constexpr int kDqWarps = 4 * kGroups;
@@ -69,10 +71,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *sC = sX + SX * slotb;
     uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
-    uint64_t *x_full = bars, *x_empty = bars + SX;
+    // stage slot g = q % 4: X slot g and TMEM A slot g share one release barrier free[g]
+    uint64_t *x_full = bars, *free_b = bars + SX;
     uint64_t *c_full = bars + 2 * SX, *c_empty = c_full + SC;
-    uint64_t *a_full = c_empty + SC, *a_empty = a_full + kGroups;
-    uint64_t *acc_full = a_empty + kGroups;
+    uint64_t *a_full = c_empty + SC;
+    uint64_t *acc_full = a_full + kGroups;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *s_level = reinterpret_cast<float *>(tmem_slot + 2);
@@ -95,10 +98,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         s_level[threadIdx.x] = v;
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&x_empty[i], 1); }
+        for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&free_b[i], 1); }
         // a chunk is read by the two groups of its two stages
         for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 8); }
-        for (int i = 0; i < kGroups; ++i) { mbar_init(&a_full[i], 8); mbar_init(&a_empty[i], 1); }
+        for (int i = 0; i < kGroups; ++i) mbar_init(&a_full[i], 8);
         mbar_init(acc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -129,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int q = 0; q < Q; ++q) {
                 const int sx = q % SX;
-                if (!mbar_wait(&x_empty[sx], ((q / SX) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait(&free_b[sx], ((q / SX) & 1) ^ 1, abort_flag)) break;
                 const uint32_t bar0 = mapa_shared(smem_u32(&x_full[sx]), 0);
                 uint8_t *slot = sX + sx * slotb;
                 if (q < QM) {
@@ -166,7 +169,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t idesc = make_idesc_bf16(2 * BM, p.BN, 0, 0);
             for (int q = 0; q < Q; ++q) {
                 const int sx = q % SX, g = q % kGroups;
-                if (!mbar_wait(&x_full[sx], (q / SX) & 1, abort_flag)) break;
                 if (!mbar_wait(&a_full[g], (q / kGroups) & 1, abort_flag)) break;
                 tc_fence_after();
                 // MMAs of this stage: 8 for a full main stage, 4 for the last odd chunk,
@@ -177,8 +179,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint64_t bdesc = make_sdesc_sw128(xbase + (kk >> 2) * xsb + (kk & 3) * 32, 16, 1024);
                     mma_ts_pair(tmem_acc, tmem_a + g * 64 + kk * 8, bdesc, idesc, (q > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit_pair(&a_empty[g]);
-                tc_commit_pair(&x_empty[sx]);
+                tc_commit_pair(&free_b[sx]);
             }
             tc_commit_pair(acc_full);
             mbar_drain(acc_full, 0);
@@ -217,7 +218,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
         for (int q = grp; q < Q && ok; q += kGroups) {
             const int g = grp;
-            if (!mbar_wait(&a_empty[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             if (q < QM) {
                 const int ci = q >> 1, sc = ci % SC;
@@ -272,6 +273,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             tmem_wait_st();
             tc_fence_before();
+            // the even CTA's warps arrive only once the stage's X tile (both halves) has landed,
+            // so a completed a_full also means a completed x_full for the MMA thread
+            if (rank == 0 && !mbar_wait(&x_full[g], (q / kGroups) & 1, abort_flag)) { ok = false; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
         }
