@@ -16,7 +16,8 @@ import torch
 from . import _capi
 
 __all__ = ["NF4Weight", "qlora_packed_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq", "qlora_dequant",
-           "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
+           "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
+           "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
            "qlora_sync_status", "QloraError"]
 
 QloraError = _capi.QloraError
@@ -111,6 +112,23 @@ def qlora_lora_linear_fwd(weight: NF4Weight, X, A, B, r: int, scaling: float, Y,
     _capi.check("qlora_lora_linear_fwd", _lib().qlora_lora_linear_fwd(
         ctypes.byref(s), _ptr(X), M, _ptr(A), _ptr(B), int(r), float(scaling), _ptr(Y), _ptr(U_save), _ptr(ws),
         wsb, _stream(stream)))
+
+
+def qlora_lora_linear_fwd_static_ws(weight: NF4Weight, X, A, B, r: int, scaling: float, Y, U_save=None,
+                                    stream=None) -> None:
+    """qlora_lora_linear_fwd with the library's static device scratch (no workspace argument)."""
+    M = X.shape[0]
+    _need(X, torch.bfloat16, (M, weight.n_in), "X")
+    _need(Y, torch.bfloat16, (M, weight.n_out), "Y")
+    if r:
+        _need(A, torch.bfloat16, (r, weight.n_in), "A")
+        _need(B, torch.bfloat16, (weight.n_out, r), "B")
+    if U_save is not None:
+        _need(U_save, torch.bfloat16, (M, r), "U_save")
+    s = weight.c_struct()
+    _capi.check("qlora_lora_linear_fwd_static_ws", _lib().qlora_lora_linear_fwd_static_ws(
+        ctypes.byref(s), _ptr(X), M, _ptr(A), _ptr(B), int(r), float(scaling), _ptr(Y), _ptr(U_save),
+        _stream(stream)))
 
 
 def qlora_lora_linear_bwd_dx(weight: NF4Weight, dY, A, B, r: int, scaling: float, dX, G_save=None, ws=None,

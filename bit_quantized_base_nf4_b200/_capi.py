@@ -8,6 +8,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqlora_nf4.so")
 
 QLORA_OK = 0
+QLORA_STATIC_SCRATCH_BYTES = 8 << 20   # the header's QLORA_STATIC_SCRATCH_BYTES
 STATUS_NAMES = {0: "QLORA_OK", 1: "QLORA_ERR_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGN",
                 4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_CUDA", 6: "QLORA_ERR_TIMEOUT",
                 7: "QLORA_ERR_UNSUPPORTED"}
@@ -30,6 +31,7 @@ SIGNATURES = {
     "qlora_dequant": (_int, [_WP, _vp, _int, _vp]),
     "qlora_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "qlora_lora_linear_fwd": (_int, [_WP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_lora_linear_fwd_static_ws": (_int, [_WP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp]),
     "qlora_lora_linear_bwd_dx": (_int, [_WP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_lora_grad_AB": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _f32, _vp, _vp, _int, _vp]),
     "qlora_sync_status": (_int, [_vp]),

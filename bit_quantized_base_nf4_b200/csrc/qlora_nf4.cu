@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 
 #include "host_common.cuh"
 #include "ptx.cuh"
@@ -13,6 +14,11 @@
 #include "fused_bwd.cuh"
 
 using namespace qlora;
+
+// Scratch of qlora_lora_linear_fwd_static_ws: part of this module's global
+// memory on every device where the module is loaded; zero-filled at load, and
+// each call clears the parts it accumulates into.
+static __device__ __align__(256) uint8_t g_static_scratch[QLORA_STATIC_SCRATCH_BYTES];
 
 namespace {
 
@@ -143,6 +149,27 @@ qlora_status check_rank(int r, float scaling, const void *A, const void *B) {
     if (!A || !B) return fail(QLORA_ERR_ARG, "A and B must be non-NULL when r > 0");
     if (!aligned16(A) || !aligned16(B)) return fail(QLORA_ERR_ALIGN, "A and B must be 16-byte aligned");
     if (!std::isfinite(scaling)) return fail(QLORA_ERR_ARG, "scaling must be finite");
+    return QLORA_OK;
+}
+
+// Device address of g_static_scratch on the current device, looked up by the
+// first call on that device and cached (one lookup per device, under a lock).
+qlora_status static_scratch(void **out) {
+    constexpr int kMaxDevices = 64;
+    static void *ptrs[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    QL_TRY(cuda_check(cudaGetDevice(&dev), "cudaGetDevice"));
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(QLORA_ERR_UNSUPPORTED, "device %d: the static scratch serves devices 0..%d", dev, kMaxDevices - 1);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        QL_TRY(cuda_check(cudaGetSymbolAddress(&p, g_static_scratch), "cudaGetSymbolAddress(static scratch)"));
+        if (!p) return fail(QLORA_ERR_CUDA, "cudaGetSymbolAddress returned NULL for the static scratch");
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
     return QLORA_OK;
 }
 
@@ -318,6 +345,26 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     QL_TRY(launch_check("fused_fwd_kernel launch"));
     if (yacc) QL_TRY(launch_finalize(yacc, M * N, 1.0f, Y, nullptr, st));
     return QLORA_OK;
+}
+
+qlora_status qlora_lora_linear_fwd_static_ws(const qlora_nf4_weight *w, const qlora_bf16 *X, int64_t M,
+                                             const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                             qlora_bf16 *Y, qlora_bf16 *U_save, void *stream) {
+    // the size check needs only host arithmetic: reject before any CUDA call
+    QL_TRY(check_weight(w));
+    if (M <= 0 || M > INT32_MAX) return fail(QLORA_ERR_SHAPE, "M (%lld) must be in [1, 2^31)", (long long)M);
+    QL_TRY(check_rank(r, scaling, A, B));
+    const size_t need = fwd_ws_bytes(M, w->n_out, w->n_in, r);
+    if (need > QLORA_STATIC_SCRATCH_BYTES)
+        return fail(QLORA_ERR_WORKSPACE,
+                    "M=%lld N=%lld K=%lld r=%d needs %zu bytes of scratch; the static scratch holds %zu "
+                    "(use qlora_lora_linear_fwd with a caller workspace)",
+                    (long long)M, (long long)w->n_out, (long long)w->n_in, r, need,
+                    size_t(QLORA_STATIC_SCRATCH_BYTES));
+    QL_TRY(require_sm100());
+    void *scratch = nullptr;
+    QL_TRY(static_scratch(&scratch));
+    return qlora_lora_linear_fwd(w, X, M, A, B, r, scaling, Y, U_save, scratch, QLORA_STATIC_SCRATCH_BYTES, stream);
 }
 
 qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf16 *dY, int64_t M, const qlora_bf16 *A,

@@ -22,7 +22,9 @@
  * Memory: every pointer is DEVICE memory owned by the caller, except where a
  * parameter says "host".  The library allocates no device memory in any
  * call; scratch space is the caller's `ws` buffer of at least
- * qlora_workspace_bytes(...) bytes.  Device pointers must be 16-byte aligned.
+ * qlora_workspace_bytes(...) bytes, except in
+ * qlora_lora_linear_fwd_static_ws, which uses a fixed scratch array held by
+ * the library.  Device pointers must be 16-byte aligned.
  *
  * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  * stream).  Calls only enqueue work; they do not synchronise.
@@ -120,6 +122,42 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
                                    const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
                                    qlora_bf16 *Y, qlora_bf16 *U_save,
                                    void *ws, size_t ws_bytes, void *stream);
+
+/* Size of the library's static device scratch used by
+ * qlora_lora_linear_fwd_static_ws: 8 MiB on each device. */
+#define QLORA_STATIC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/* The forward of qlora_lora_linear_fwd (same arguments, same kernels, same
+ * results) with no ws / ws_bytes: its scratch is a file-scope
+ * `__device__` array of QLORA_STATIC_SCRATCH_BYTES that the library's module
+ * holds on every device where it is loaded.  The QLoRA paper has no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory for a workspace: a plain-C host that is handed only the
+ * layer's tensors and has no allocator of its own; a process whose free
+ * device memory is already reserved by a caching allocator (torch's, for
+ * one), where a cudaMalloc of its own fails with out-of-memory; and a loop
+ * in which cudaFree's implicit device synchronisation would stall the
+ * other streams.  This call makes no cudaMalloc, cudaFree or other
+ * allocating call.
+ *   Set-up: the first call on each device, with that device current, looks
+ *   up the array's device address (cudaGetSymbolAddress) and keeps it for
+ *   later calls; a failure of that lookup returns QLORA_ERR_CUDA.  Make
+ *   this first call on a device before any stream capture.
+ *   Limit: when the forward's scratch need for these sizes (the rank-r
+ *   buffers, about 6 * M * r bytes, plus a 4 * M * N byte split-K
+ *   accumulator when M < 64 and K is split) exceeds
+ *   QLORA_STATIC_SCRATCH_BYTES, the call
+ *   returns QLORA_ERR_WORKSPACE before touching the device; use
+ *   qlora_lora_linear_fwd with a caller workspace instead.
+ *   Zeroing: the fp32 accumulators in the scratch are cleared on `stream`
+ *   by every call before its kernels add into them.
+ *   Concurrency: every call on a device uses the same scratch, so two calls
+ *   whose work overlaps in time (different streams, or host threads with no
+ *   ordering between their streams) race and give wrong results; order them
+ *   on one stream or with events. */
+qlora_status qlora_lora_linear_fwd_static_ws(const qlora_nf4_weight *w, const qlora_bf16 *X, int64_t M,
+                                             const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                             qlora_bf16 *Y, qlora_bf16 *U_save, void *stream);
 
 /* Backward to the input: dX = dY W' + scaling * (dY B) A  (the frozen base
  * is a read-only operator; no gradient is formed for W0).
