@@ -159,6 +159,26 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
     return d;
 }
 
+// As make_sdesc_sw128 for any swizzle span: 32, 64 or 128 bytes (layout codes 6, 4, 2;
+// atoms aligned to 256, 512 and 1024 bytes respectively).
+__device__ __forceinline__ uint64_t make_sdesc_swz(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                                   uint32_t span_bytes) {
+    const uint64_t layout = span_bytes == 128 ? 2 : (span_bytes == 64 ? 4 : 6);
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;
+    d |= layout << 61;
+    return d;
+}
+
+// Four fp32 atomic adds to 16 consecutive, 16-byte aligned bytes (no return value).
+__device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 // 32 lanes x 32-bit, 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(

@@ -111,28 +111,64 @@ size_t bwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
     return ws_layout(M, K, r, plan_gemm(M, K, ceil_div(N, 64)).splits > 1).total;
 }
 
-// Launches the rank-r tensor-core product (see skinny_mma.cuh); the output must
-// already hold zeros or the values to accumulate into.
-qlora_status launch_skinny(const CUtensorMap &tmA, const CUtensorMap &tmB, int a_mn, int b_mn, int64_t T, int64_t I,
-                           int r, float scaling, float *out, int64_t ld_row, int64_t ld_col, cudaStream_t st) {
-    const int64_t ST = ceil_div(T, 64);
-    const int64_t tiles = ceil_div(I, skinny::BI);
-    const int64_t want = std::max<int64_t>(1, ceil_div(2 * sm_count(), tiles));
-    const int64_t sps = ceil_div(ST, std::min(ST, want));
-    skinny::Params p;
+// Launches the rank-r tensor-core product out[i*ld_i + j*ld_j] += scaling *
+// sum_t P(i, t) Q(j, t) (see skinny_mma.cuh) over bf16 operands:
+//   P: p_mn = 0 -> [I, T] row-major (t contiguous); p_mn = 1 -> [T, I] row-major
+//   Q: q_mn = 0 -> [r, T] row-major;                q_mn = 1 -> [T, r] row-major
+// The output must already hold zeros or the values to accumulate into.
+qlora_status launch_skinny(const void *P, int p_mn, const void *Q, int q_mn, int64_t T, int64_t I, int r,
+                           float scaling, float *out, int64_t ld_i, int64_t ld_j, cudaStream_t st) {
+    using namespace skinny;
+    Params p;
     p.T = static_cast<int>(T);
     p.I = static_cast<int>(I);
     p.r = r;
-    p.stages_per_split = static_cast<int>(sps);
-    p.a_mn = a_mn;
-    p.b_mn = b_mn;
+    p.p_mn = p_mn;
+    p.q_mn = q_mn;
+    CUtensorMap tmP, tmQ;
+    // P: one 3-D box per stage when the t (K-major) or i (MN-major) extent is whole 64-element chunks
+    const int64_t p_rows = p_mn ? T : I, p_cols = p_mn ? I : T;
+    p.p_3d = p_cols % 64 == 0;
+    if (p.p_3d)
+        QL_TRY(make_tmap_chunks(&tmP, P, p_rows, p_cols, BT, 2));
+    else
+        QL_TRY(make_tmap_2d(&tmP, P, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p_rows, p_cols, p_cols, BT, 64,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+    if (!q_mn) {
+        // [r, T]: Nq rows per 64-t chunk, rows past r zero-filled
+        p.Nq = static_cast<int>(ceil_div(r, 16) * 16);
+        p.q_3d = T % 64 == 0;
+        p.q_atoms = 0;
+        p.q_span = 128;
+        p.q_bytes = 2 * p.Nq * 128;
+        if (p.q_3d)
+            QL_TRY(make_tmap_chunks(&tmQ, Q, r, T, p.Nq, 2));
+        else
+            QL_TRY(make_tmap_2d(&tmQ, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, T, T, p.Nq, 64,
+                                CU_TENSOR_MAP_SWIZZLE_128B));
+    } else {
+        // [T, r]: j contiguous; the narrowest swizzle atom that covers r (16, 32 or 64 elements)
+        p.Nq = r <= 16 ? 16 : (r <= 32 ? 32 : (r <= 64 ? 64 : 128));
+        p.q_span = p.Nq >= 64 ? 128 : p.Nq * 2;
+        p.q_atoms = p.Nq >= 64 ? p.Nq / 64 : 1;
+        p.q_3d = 0;
+        p.q_bytes = p.q_atoms * BT * p.q_span;
+        const CUtensorMapSwizzle swz = p.q_span == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                       : p.q_span == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                        : CU_TENSOR_MAP_SWIZZLE_32B;
+        QL_TRY(make_tmap_2d(&tmQ, Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, r, r, BT, p.q_span / 2, swz));
+    }
+    p.stages = std::min(kMaxStages, kRingBudget / stage_bytes(p.q_bytes));
+    p.units = ceil_div(I, BI) * ceil_div(T, BT);
     p.scaling = scaling;
     p.out = out;
-    p.ld_row = ld_row;
-    p.ld_col = ld_col;
-    QL_TRY(set_smem(skinny::skinny_mma_kernel, skinny::smem_bytes()));
-    dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(ceil_div(ST, sps)));
-    skinny::skinny_mma_kernel<<<grid, skinny::kThreads, skinny::smem_bytes(), st>>>(tmA, tmB, p);
+    p.ld_i = ld_i;
+    p.ld_j = ld_j;
+    const int smem = smem_bytes(p.stages, p.q_bytes);
+    QL_TRY(set_smem(skinny_mma_kernel, smem));
+    // stream-K: one CTA per SM, each a contiguous run of (tile, stage) units
+    const int64_t grid = std::min<int64_t>(p.units, sm_count());
+    skinny_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tmP, tmQ, p);
     return launch_check("skinny_mma_kernel launch");
 }
 
@@ -274,12 +310,9 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     float *uacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
     float *yacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
     if (r > 0) {
-        // U^T = A . X^T on tensor cores, then bf16 copies: U (saved) and scaling * U (adapter chunk)
-        CUtensorMap tA, tB;
-        QL_TRY(make_tmap_2d(&tA, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, r, K, K, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-        QL_TRY(make_tmap_2d(&tB, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, 256, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        // U = X A^T on tensor cores, then bf16 copies: U (saved) and scaling * U (adapter chunk)
         QL_TRY(cuda_check(cudaMemsetAsync(uacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
-        QL_TRY(launch_skinny(tA, tB, 0, 0, K, M, r, 1.0f, uacc, 1, r, st));
+        QL_TRY(launch_skinny(X, 0, A, 0, K, M, r, 1.0f, uacc, r, 1, st));
         QL_TRY(launch_finalize(uacc, M * r, scaling, U_save, us, st));
     }
     const Codebook &cb = codebook();
@@ -390,12 +423,9 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     float *gacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
     float *dxacc = g.splits > 1 ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
     if (r > 0) {
-        // G^T = B^T . dY^T on tensor cores (B read MN-major), then bf16 copies G and scaling * G
-        CUtensorMap tA, tB;
-        QL_TRY(make_tmap_2d(&tA, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-        QL_TRY(make_tmap_2d(&tB, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, 256, 64, CU_TENSOR_MAP_SWIZZLE_128B));
+        // G = dY B on tensor cores (B read MN-major), then bf16 copies G and scaling * G
         QL_TRY(cuda_check(cudaMemsetAsync(gacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
-        QL_TRY(launch_skinny(tA, tB, 1, 0, N, M, r, 1.0f, gacc, 1, r, st));
+        QL_TRY(launch_skinny(dY, 0, B, 1, N, M, r, 1.0f, gacc, r, 1, st));
         QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
     }
     if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
@@ -455,14 +485,9 @@ qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const
         QL_TRY(cuda_check(cudaMemsetAsync(dA, 0, size_t(r) * K * 4, st), "zero dA"));
         QL_TRY(cuda_check(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, st), "zero dB"));
     }
-    // dA [r, K] = s G^T X  and  dB^T [r, N] = s U^T dY, contraction over the M tokens
-    CUtensorMap tG, tX, tU, tY;
-    QL_TRY(make_tmap_2d(&tG, G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(make_tmap_2d(&tX, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(make_tmap_2d(&tU, U, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(make_tmap_2d(&tY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(launch_skinny(tG, tX, 1, 1, M, K, r, scaling, dA, K, 1, st));
-    QL_TRY(launch_skinny(tU, tY, 1, 1, M, N, r, scaling, dB, 1, r, st));
+    // dA^T [K, r] = s X^T G  and  dB [N, r] = s dY^T U, contraction over the M tokens
+    QL_TRY(launch_skinny(X, 1, G, 1, M, K, r, scaling, dA, 1, K, st));
+    QL_TRY(launch_skinny(dY, 1, U, 1, M, N, r, scaling, dB, r, 1, st));
     return QLORA_OK;
 }
 

@@ -1,18 +1,24 @@
 // skinny_mma.cuh -- the rank-r products of the adapter on tcgen05 tensor cores.
 //
-//   D[j, i] = sum_t Aop(j, t) * Bop(i, t),   j < r (MMA M = 128, rows past r are zero),
-//                                             i in tiles of 256 (MMA N), t split across CTAs
-//   out[j * ld_row + i * ld_col] += scaling * D[j, i]      (fp32 atomics)
+//   D[i, j] = sum_t P(i, t) * Q(j, t),    i in tiles of 128 (MMA M = TMEM lanes),
+//                                          j < r (MMA N = Nq, a multiple of 16 >= r),
+//                                          t in stages of 128
+//   out[i * ld_i + j * ld_j] += scaling * D[i, j]      (fp32 reductions)
 //
-// with the operand of each side either K-major (t contiguous, a [rows, t] tensor)
-// or MN-major (rows contiguous, a [t, rows] tensor), both staged by TMA in the
-// 128-byte-swizzled layouts the MMA reads directly:
-//   U^T = A_lora . X^T     Aop = A [r, K] K-major,        Bop = X [M, K] K-major
-//   G^T = B_lora^T . dY^T  Aop = B [N, r] MN-major,       Bop = dY [M, N] K-major
-//   dA  = G^T . X          Aop = G [M, r] MN-major,       Bop = X [M, K] MN-major
-//   dB^T = U^T . dY        Aop = U [M, r] MN-major,       Bop = dY [M, N] MN-major
-// These products stream the activation once from HBM; the tensor core keeps
-// them memory-bound at any adapter rank up to 128.
+// P is the streamed activation, Q the small rank-r factor; each is K-major (t
+// contiguous) or MN-major (i or j contiguous) and is staged by TMA in the
+// swizzled layout the MMA reads directly:
+//   U  = X . A_lora^T   P = X [M, K] K-major,    Q = A [r, K] K-major,   out [M, r]
+//   G  = dY . B_lora    P = dY [M, N] K-major,   Q = B [N, r] MN-major,  out [M, r]
+//   dA^T = X^T . G      P = X [M, K] MN-major,   Q = G [M, r] MN-major,  out dA [r, K]
+//   dB = dY^T . U       P = dY [M, N] MN-major,  Q = U [M, r] MN-major,  out dB [N, r]
+// The products stream P once from HBM and are memory-bound.  Putting i on the
+// TMEM lanes gives every epilogue thread one output row, so the r results of a
+// row leave in a few vector reductions.
+// Work split (stream-K): the (i tile, t stage) units are numbered tile-major and
+// each CTA takes one contiguous range of them, so every SM streams about the
+// same number of bytes; the accumulator is double-buffered in TMEM so the
+// epilogue of one tile overlaps the MMAs of the next.
 #pragma once
 
 #include <cstdint>
@@ -23,51 +29,65 @@
 namespace qlora {
 namespace skinny {
 
-constexpr int BI = 256;                  // columns i per tile (MMA N)
-constexpr int SXS = 4;                   // pipeline stages (64 t each)
-constexpr int kThreads = 256;            // warp 0 TMA, 1 MMA, 2 TMEM alloc, 4-7 epilogue
-constexpr int kAStage = 128 * 128;       // 128 rows x 64 t bf16
-constexpr int kBStage = BI * 128;        // 256 rows x 64 t bf16
-constexpr int kStage = kAStage + kBStage;
+constexpr int BI = 128;                    // i per tile
+constexpr int BT = 128;                    // t per stage
+constexpr int kThreads = 192;              // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int kPBytes = BI * BT * 2;       // 32 KB
+constexpr int kMaxStages = 8;
+constexpr int kRingBudget = 200 * 1024;    // bytes of stage buffers
+constexpr int kTmemCols = 256;             // two accumulators of up to 128 columns
 
 struct Params {
-    int T;                 // contraction length
-    int I;                 // number of columns
-    int r;                 // valid rows
-    int stages_per_split;  // 64-wide t stages per CTA along blockIdx.y
-    int a_mn, b_mn;        // operand majorness (0: K-major, 1: MN-major)
+    int T;             // contraction length
+    int I;             // rows i
+    int r;             // valid columns j
+    int Nq;            // MMA N: multiple of 16, r <= Nq <= 128
+    int p_mn, q_mn;    // majorness (0: K-major, 1: MN-major)
+    int p_3d;          // P as one 3-D box {64, 128, 2} (else two 2-D boxes of 64 x 128)
+    int q_3d;          // K-major Q as one 3-D box {64, Nq, 2} (else two 2-D boxes)
+    int q_atoms;       // MN-major Q: swizzle atoms per stage (1 or 2)
+    int q_span;        // MN-major Q: swizzle span in bytes (32, 64 or 128) = row bytes of an atom
+    int q_bytes;       // Q bytes per stage
+    int stages;        // ring depth
+    int64_t units;     // tiles * stages along t
     float scaling;
     float *out;
-    int64_t ld_row, ld_col;
+    int64_t ld_i, ld_j;
 };
 
-__host__ __device__ constexpr int smem_bytes() { return 1024 + SXS * kStage + 512; }
+__host__ __device__ constexpr int stage_bytes(int q_bytes) { return kPBytes + q_bytes; }
+__host__ __device__ constexpr int smem_bytes(int stages, int q_bytes) {
+    return 1024 + stages * stage_bytes(q_bytes) + 256;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
-    skinny_mma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    skinny_mma_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                       const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SXS * kStage);
-    uint64_t *full = bars, *empty = bars + SXS, *acc_full = bars + 2 * SXS;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    const int SB = stage_bytes(p.q_bytes);
+    const int S = p.stages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * SB);
+    uint64_t *full = bars, *empty = bars + kMaxStages;
+    uint64_t *acc_full = bars + 2 * kMaxStages, *acc_empty = acc_full + 2, *mma_done = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int i0 = blockIdx.x * BI;
-    const int ST = (p.T + 63) / 64;
-    const int s_begin = blockIdx.y * p.stages_per_split;
-    const int s_end = min(ST, s_begin + p.stages_per_split);
-    const int nst = s_end - s_begin;
+    const int ST = (p.T + BT - 1) / BT;
+    const int64_t u_begin = p.units * blockIdx.x / gridDim.x;
+    const int64_t u_end = p.units * (blockIdx.x + 1) / gridDim.x;
+    const int nu = static_cast<int>(u_end - u_begin);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < SXS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        mbar_init(acc_full, 1);
+        for (int i = 0; i < S; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+        mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 2) {
-        tmem_alloc(tmem_slot, 256);
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -76,84 +96,133 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0 && nst > 0) {
-            tma_prefetch_desc(&tmA);
-            tma_prefetch_desc(&tmB);
+        if (lane == 0 && nu > 0) {
+            tma_prefetch_desc(&tmP);
+            tma_prefetch_desc(&tmQ);
+            const uint32_t tx = kPBytes + p.q_bytes;
+            const int qw = p.q_span / 2;          // elements per MN-major Q atom row
             int issued = 0;
-            for (int s = 0; s < nst; ++s) {
-                const int sx = s % SXS;
-                if (!mbar_wait(&empty[sx], ((s / SXS) & 1) ^ 1, abort_flag)) break;
-                uint8_t *sa = smem + sx * kStage;
-                uint8_t *sb = sa + kAStage;
-                const int t0 = (s_begin + s) * 64;
-                mbar_arrive_expect_tx(&full[sx], kStage);
-                if (p.a_mn) {
-                    tma_load_2d(sa, &tmA, &full[sx], 0, t0);
-                    tma_load_2d(sa + 8192, &tmA, &full[sx], 64, t0);
-                } else {
-                    tma_load_2d(sa, &tmA, &full[sx], t0, 0);
+            for (int k = 0; k < nu; ++k) {
+                const int64_t u = u_begin + k;
+                const int i0 = static_cast<int>(u / ST) * BI;
+                const int t0 = static_cast<int>(u % ST) * BT;
+                const int sx = k % S;
+                if (!mbar_wait(&empty[sx], ((k / S) & 1) ^ 1, abort_flag)) break;
+                uint8_t *sp = smem + sx * SB;
+                uint8_t *sq = sp + kPBytes;
+                mbar_arrive_expect_tx(&full[sx], tx);
+                if (!p.p_mn) {                     // [I, T]: rows i, t contiguous
+                    if (p.p_3d) {
+                        tma_load_3d(sp, &tmP, &full[sx], 0, i0, t0 / 64);
+                    } else {
+                        tma_load_2d(sp, &tmP, &full[sx], t0, i0);
+                        tma_load_2d(sp + kPBytes / 2, &tmP, &full[sx], t0 + 64, i0);
+                    }
+                } else {                           // [T, I]: rows t, i contiguous
+                    if (p.p_3d) {
+                        tma_load_3d(sp, &tmP, &full[sx], 0, t0, i0 / 64);
+                    } else {
+                        tma_load_2d(sp, &tmP, &full[sx], i0, t0);
+                        tma_load_2d(sp + kPBytes / 2, &tmP, &full[sx], i0 + 64, t0);
+                    }
                 }
-                if (p.b_mn) {
-#pragma unroll
-                    for (int q = 0; q < BI / 64; ++q) tma_load_2d(sb + 8192 * q, &tmB, &full[sx], i0 + 64 * q, t0);
-                } else {
-                    tma_load_2d(sb, &tmB, &full[sx], t0, i0);
+                if (!p.q_mn) {                     // [r, T]
+                    if (p.q_3d) {
+                        tma_load_3d(sq, &tmQ, &full[sx], 0, 0, t0 / 64);
+                    } else {
+                        tma_load_2d(sq, &tmQ, &full[sx], t0, 0);
+                        tma_load_2d(sq + p.Nq * 128, &tmQ, &full[sx], t0 + 64, 0);
+                    }
+                } else {                           // [T, r]
+                    for (int a = 0; a < p.q_atoms; ++a)
+                        tma_load_2d(sq + a * BT * p.q_span, &tmQ, &full[sx], a * qw, t0);
                 }
-                issued = s + 1;
+                issued = k + 1;
             }
-            for (int s = max(0, issued - SXS); s < issued; ++s) mbar_drain(&full[s % SXS], (s / SXS) & 1);
+            for (int k = max(0, issued - S); k < issued; ++k) mbar_drain(&full[k % S], (k / S) & 1);
         }
     } else if (warp == 1) {
-        if (lane == 0 && nst > 0) {
-            const uint32_t idesc = make_idesc_bf16(128, BI, p.a_mn, p.b_mn);
-            for (int s = 0; s < nst; ++s) {
-                const int sx = s % SXS;
-                if (!mbar_wait(&full[sx], (s / SXS) & 1, abort_flag)) break;
+        if (lane == 0 && nu > 0) {
+            const uint32_t idesc = make_idesc_bf16(BI, p.Nq, p.p_mn, p.q_mn);
+            int seg = 0;
+            for (int k = 0; k < nu; ++k) {
+                const int64_t u = u_begin + k;
+                const bool first = (k == 0) || (u % ST == 0);
+                const bool last = (k == nu - 1) || ((u + 1) % ST == 0);
+                const int buf = seg & 1;
+                if (first && !mbar_wait(&acc_empty[buf], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+                const int sx = k % S;
+                if (!mbar_wait(&full[sx], (k / S) & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t sa = smem_u32(smem + sx * kStage);
-                const uint32_t sb = sa + kAStage;
+                const uint32_t sp = smem_u32(smem + sx * SB);
+                const uint32_t sq = sp + kPBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = p.a_mn ? make_sdesc_sw128(sa + kk * 2048, 8192, 1024)
-                                               : make_sdesc_sw128(sa + kk * 32, 16, 1024);
-                    const uint64_t bd = p.b_mn ? make_sdesc_sw128(sb + kk * 2048, 8192, 1024)
-                                               : make_sdesc_sw128(sb + kk * 32, 16, 1024);
-                    mma_ss(tmem, ad, bd, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < BT / 16; ++kk) {
+                    const uint64_t pd = p.p_mn ? make_sdesc_sw128(sp + kk * 2048, kPBytes / 2, 1024)
+                                               : make_sdesc_sw128(sp + (kk >> 2) * (kPBytes / 2) + (kk & 3) * 32,
+                                                                  16, 1024);
+                    const uint64_t qd =
+                        p.q_mn ? make_sdesc_swz(sq + kk * 16 * p.q_span, BT * p.q_span, 8 * p.q_span, p.q_span)
+                               : make_sdesc_sw128(sq + (kk >> 2) * (p.Nq * 128) + (kk & 3) * 32, 16, 1024);
+                    mma_ss(tmem + buf * 128, pd, qd, idesc, (first && kk == 0) ? 0u : 1u);
                 }
                 tc_commit(&empty[sx]);
+                if (last) {
+                    tc_commit(&acc_full[buf]);
+                    ++seg;
+                }
             }
-            tc_commit(acc_full);
-            mbar_drain(acc_full, 0);
+            // TMEM is released only after every MMA has completed
+            tc_commit(mma_done);
+            mbar_drain(mma_done, 0);
         }
-    } else if (warp >= 4 && nst > 0) {
+    } else if (nu > 0) {
+        // epilogue, warps 2-5: TMEM lane quadrant (warp % 4), one output row i per thread
         const int quad = warp & 3;
-        if (quad * 32 < p.r && mbar_wait(acc_full, 0, abort_flag)) {
+        const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        int seg = 0;
+        for (int k = 0; k < nu; ++k) {
+            const int64_t u = u_begin + k;
+            const bool last = (k == nu - 1) || ((u + 1) % ST == 0);
+            if (!last) continue;
+            const int buf = seg & 1;
+            const int i = static_cast<int>(u / ST) * BI + quad * 32 + lane;
+            if (!mbar_wait(&acc_full[buf], (seg >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const int j = quad * 32 + lane;
-            const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16);
-            for (int ch = 0; ch < BI / 16; ++ch) {
-                if (i0 + ch * 16 >= p.I) break;   // warp-uniform
+            for (int c = 0; c < p.r; c += 16) {
                 uint32_t v[16];
-                tmem_ld16(taddr + ch * 16, v);
+                tmem_ld16(tmem + lane_addr + buf * 128 + c, v);
                 tmem_wait_ld16(v);
-                if (j < p.r) {
+                if (i < p.I) {
+                    if (p.ld_j == 1) {             // row i holds r consecutive floats: 16-byte reductions
+                        float *dst = p.out + int64_t(i) * p.ld_i + c;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int i = i0 + ch * 16 + e;
-                        if (i < p.I)
-                            atomicAdd(p.out + int64_t(j) * p.ld_row + int64_t(i) * p.ld_col,
-                                      p.scaling * __uint_as_float(v[e]));
+                        for (int q = 0; q < 4; ++q)
+                            if (c + 4 * q < p.r)
+                                red_add_v4(dst + 4 * q, p.scaling * __uint_as_float(v[4 * q]),
+                                           p.scaling * __uint_as_float(v[4 * q + 1]),
+                                           p.scaling * __uint_as_float(v[4 * q + 2]),
+                                           p.scaling * __uint_as_float(v[4 * q + 3]));
+                    } else {                       // ld_i == 1: the warp's 32 rows are contiguous
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c + e < p.r)
+                                atomicAdd(p.out + int64_t(c + e) * p.ld_j + i, p.scaling * __uint_as_float(v[e]));
                     }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            ++seg;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
