@@ -1,0 +1,313 @@
+// fused_bwd_pair.cuh -- input-gradient GEMM with NF4 dequant, on CTA pairs (tcgen05 cta_group::2).
+//
+//   D[k, m] = sum_n W'[n, k] dY[m, n]  +  sum_j A[j, k] gs[m, j]     k in 256 columns of W0
+//                                                                      (128 per CTA), m in BN tokens
+// with gs = bf16(scaling * dY B) from the rank-r side kernel; dX = D^T.
+//
+// Two CTAs on two SMs form one 256-k x BN-token tile.  Each CTA dequantizes the
+// weight for its own 128 k into its own shared memory, as the MN-major
+// (k contiguous) 128-byte-swizzled A operand, and loads only its half of the
+// token tile (BN/2 rows of dY); one tcgen05.mma.cta_group::2 issued by the even
+// CTA reads both CTAs' A halves and B halves.
+//
+// The MMA issue is effectively synchronous with the issuing thread, so the MMA
+// thread does one barrier wait and one commit per stage of 64 n (four MMAs of
+// 256 x BN x 16): it waits on a_full[s % 4], which the even CTA's dequant warps
+// arrive on only after they have seen the stage's dY tile land, and commits to
+// free[s % 4], which releases the dY slot and the A slot of the stage in both CTAs.
+//   producer (warp 0)    one TMA instruction per stage: this CTA's dY half,
+//                        counted on the even CTA's y_full
+//   producer (warp 3)    packed codes, 256 n rows x 128 k (four stages) per TMA
+//                        instruction
+//   dequant group s % 4  (4 warps, thread = one 64-block: a row n and a 64-k half)
+//                        expands the block through a byte -> (level[lo], level[hi])
+//                        bf16x2 table times the bf16 block scale, stores it
+//                        swizzled into A slot s % 4, then arrives on a_full
+//   MMA (warp 1, even)   four tcgen05.mma (K = 16), A and B from shared memory
+// Commits are multicast to both CTAs (free, acc_full); each CTA then reads back
+// its own 128 x BN accumulator and writes dX.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace qlora {
+namespace bwdp {
+
+constexpr int BM = 128;                       // k columns of W0 per CTA (256 per pair)
+constexpr int S = 4;                          // stage slots: dY ring = A ring = dequant groups
+constexpr int kGroups = S;
+constexpr int SC = 2;                         // code ring chunks (four stages each)
+constexpr int kDqWarps = 4 * kGroups;
+constexpr int kThreads = 128 + 32 * kDqWarps;
+constexpr int kChunkRows = 256;               // n rows per code chunk
+constexpr int kCodeChunkBytes = kChunkRows * 64;   // 64 bytes = 128 k per row
+constexpr int kAStageBytes = 64 * BM * 2;     // 64 n x 128 k bf16
+constexpr int kLutWords = 256 * 32;
+
+struct Params {
+    const uint8_t *scales;
+    const float *scales2;
+    const uint16_t *Alora;   // [r, K] bf16 or nullptr
+    uint16_t *dX;            // [M, K] bf16
+    int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
+    float level[16];
+};
+
+__host__ __device__ constexpr int smem_bytes(int BN) {
+    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes + kLutWords * 4 + 512;
+}
+__host__ __device__ constexpr uint32_t tmem_cols(int BN) {
+    return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    fused_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmC,
+                          const __grid_constant__ CUtensorMap tmG, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int half_bn = p.BN / 2;
+    const int ysb = half_bn * 128;                // this CTA's dY half for one stage
+    uint8_t *sY = smem;
+    uint8_t *sA = sY + S * ysb;
+    uint8_t *sC = sA + S * kAStageBytes;
+    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
+    uint64_t *y_full = bars, *free_b = bars + S;
+    uint64_t *c_full = bars + 2 * S, *c_empty = c_full + SC;
+    uint64_t *a_full = c_empty + SC;
+    uint64_t *acc_full = a_full + S;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *s_level = reinterpret_cast<float *>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();      // 0: even CTA (issues the MMAs), 1: its peer
+    const int k0 = blockIdx.x * BM;               // blockIdx.x = 2 * pair + rank
+    const int m0 = blockIdx.y * p.BN;
+    const int my_m0 = m0 + int(rank) * half_bn;
+    const int KB = p.K / 64;
+    const int NB = (p.N + 63) / 64;               // main stages (64 n each)
+    const int LS = p.r > 0 ? (p.r + 63) / 64 : 0; // adapter stages (64 j each)
+    const int total = NB + LS;
+    const int nchunk = (NB + 3) / 4;
+    const uint32_t ncols = tmem_cols(p.BN);
+
+    if (threadIdx.x < 16) {
+        float v = 0.f;  // constant-index reads keep the parameter block out of local memory
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if (threadIdx.x == i) v = p.level[i];
+        s_level[threadIdx.x] = v;
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&y_full[i], 1);
+            mbar_init(&free_b[i], 1);
+            mbar_init(&a_full[i], 8);             // 4 warps x 2 CTAs
+        }
+        // a chunk is read by the four groups of its four stages
+        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 4 * kGroups); }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(tmem_slot, ncols);
+        tmem_relinquish_pair();
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
+        const int e = i >> 5;
+        __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
+        sLut[i] = *reinterpret_cast<uint32_t *>(&v);
+    }
+    tc_fence_before();
+    // both CTAs' barriers are initialised before either signals the other's
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_acc = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- dY producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmY);
+            if (LS) tma_prefetch_desc(&tmG);
+            int issued = 0;
+            for (int s = 0; s < total; ++s) {
+                const int sx = s % S;
+                if (!mbar_wait(&free_b[sx], ((s / S) & 1) ^ 1, abort_flag)) break;
+                const uint32_t bar0 = mapa_shared(smem_u32(&y_full[sx]), 0);
+                if (rank == 0) mbar_arrive_expect_tx(&y_full[sx], 2 * ysb);
+                if (s < NB)
+                    tma_load_2d_pair(sY + sx * ysb, &tmY, bar0, s * 64, my_m0);
+                else
+                    tma_load_2d_pair(sY + sx * ysb, &tmG, bar0, (s - NB) * 64, my_m0);
+                issued = s + 1;
+            }
+            // the even CTA sees both CTAs' copies complete on its barriers
+            if (rank == 0)
+                for (int s = max(0, issued - S); s < issued; ++s) mbar_drain(&y_full[s % S], (s / S) & 1);
+        }
+    } else if (warp == 3) {
+        // ---------------- packed-code producer (local to each CTA)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmC);
+            int issued = 0;
+            for (int c = 0; c < nchunk; ++c) {
+                const int sc = c % SC;
+                if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&c_full[sc], kCodeChunkBytes);
+                // rows n = 256c .., bytes k0/2 .. k0/2 + 63
+                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], k0 / 2, c * kChunkRows);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (even CTA only)
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = make_idesc_bf16(2 * BM, p.BN, 1, 0);
+            for (int s = 0; s < total; ++s) {
+                const int g = s % S;
+                if (!mbar_wait_cluster(&a_full[g], (s / S) & 1, abort_flag)) break;
+                tc_fence_after();
+                const int nk = (s < NB) ? 4 : min(4, (p.r - (s - NB) * 64 + 15) / 16);
+                const uint32_t ybase = smem_u32(sY + g * ysb);
+                const uint32_t abase = smem_u32(sA + g * kAStageBytes);
+                for (int kk = 0; kk < nk; ++kk) {
+                    const uint64_t adesc = make_sdesc_sw128(abase + kk * 2048, 8192, 1024);
+                    const uint64_t bdesc = make_sdesc_sw128(ybase + kk * 32, 16, 1024);
+                    mma_ss_pair(tmem_acc, adesc, bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit_pair(&free_b[g]);
+            }
+            tc_commit_pair(acc_full);
+            mbar_drain(acc_full, 0);
+        }
+    } else if (warp >= 4) {
+        // thread = (contraction row nl, k half h): one 64-block of W0 row n
+        const int dw = warp - 4;
+        const int grp = dw >> 2;                    // stages s with s % kGroups == grp
+        const int wi = dw & 3;
+        const int nl = (wi & 1) * 32 + lane;        // contraction row within the stage (0..63)
+        const int h = wi >> 1;                      // k half: columns k0 + 64h ..
+        const int kblk = k0 / 64 + h;               // 64-block index along the row
+        const bool kvalid = kblk < KB;
+        const uint32_t lut = smem_u32(sLut) + lane * 4;
+        const uint32_t sAu = smem_u32(sA);
+        // 64-byte code rows, 64-byte swizzle: 16-byte chunk c of row q sits at chunk c ^ ((q >> 1) & 3);
+        // stage rows start at multiples of 64, so the phase depends on nl only
+        const uint32_t c_swz = (nl >> 1) & 3;
+        const uint32_t a_off = h * 8192 + nl * 128;
+        bool ok = true;
+
+        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
+            const int n = s * 64 + nl;
+            qv = 0;
+            dv = 0.f;
+            if (kvalid && s < NB && n < p.N) {
+                const int64_t b = int64_t(n) * KB + kblk;
+                qv = __ldg(p.scales + b);
+                dv = __ldg(p.scales2 + (b >> 8));
+            }
+        };
+        // block scales of this group's next three stages
+        uint32_t qa, qb, qc;
+        float da, db, dc;
+        load_scale(grp, qa, da);
+        load_scale(grp + kGroups, qb, db);
+        load_scale(grp + 2 * kGroups, qc, dc);
+
+        for (int s = grp; s < total && ok; s += kGroups) {
+            const int g = grp;
+            uint32_t out[32];
+            if (s < NB) {
+                const int ci = s >> 2, sc = ci % SC;
+                if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
+                const float sv = __fmul_rn(static_cast<float>(qa), da);
+                qa = qb; da = db; qb = qc; db = dc;
+                load_scale(s + 3 * kGroups, qc, dc);
+                __nv_bfloat162 s2b = __float2bfloat162_rn(sv);
+                const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
+                const uint32_t cbase = smem_u32(sC) + sc * kCodeChunkBytes + ((s & 3) * 64 + nl) * 64;
+                const uint4 c0 = lds128(cbase + (((2u * h + 0u) ^ c_swz) << 4));
+                const uint4 c1 = lds128(cbase + (((2u * h + 1u) ^ c_swz) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                for (int w8 = 0; w8 < 8; ++w8) {
+#pragma unroll
+                    for (int by = 0; by < 4; ++by) {
+                        const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
+                        out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                    }
+                }
+            } else {
+                // adapter chunk: row j of A [r, K], 64 k starting at k0 + 64h (zero past r / K)
+                const int j = (s - NB) * 64 + nl;
+                const int kk0 = k0 + h * 64;
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if (j < p.r && kk0 < p.K)
+                        w = __ldg(reinterpret_cast<const uint4 *>(p.Alora + int64_t(j) * p.K + kk0 + v * 8));
+                    out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
+                }
+            }
+            // A slot g is free once the MMAs of stage s - 4 have completed
+            if (!mbar_wait(&free_b[g], ((s / S) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            const uint32_t abase = sAu + g * kAStageBytes + a_off;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t chunk = uint32_t(i) ^ uint32_t(nl & 7);
+                sts128(abase + (chunk << 4), make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]));
+            }
+            fence_proxy_async_smem();
+            // the even CTA's warps arrive only once the stage's dY tile (both halves) has landed,
+            // so a completed a_full also means a completed y_full for the MMA thread
+            if (rank == 0 && !mbar_wait(&y_full[g], (s / S) & 1, abort_flag)) { ok = false; break; }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
+        }
+
+        // ---------------- epilogue: this CTA's 128 k rows x BN tokens
+        if (ok && mbar_wait(acc_full, 0, abort_flag)) {
+            tc_fence_after();
+            const int quad = warp & 3;
+            const int row = quad * 32 + lane;
+            const int k = k0 + row;
+            const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+            const int nchunks = p.BN / 16;
+            for (int ch = grp; ch < nchunks; ch += kGroups) {
+                uint32_t v[16];
+                tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
+                tmem_wait_ld16(v);
+                if (k < p.K) {
+                    const int mb = m0 + ch * 16;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (mb + i < p.M) {
+                            __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
+                            p.dX[int64_t(mb + i) * p.K + k] = *reinterpret_cast<uint16_t *>(&hv);
+                        }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // neither CTA leaves (or frees TMEM) while the pair may still touch its memory
+    cluster_sync();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_acc, ncols);
+    }
+}
+
+}  // namespace bwdp
+}  // namespace qlora

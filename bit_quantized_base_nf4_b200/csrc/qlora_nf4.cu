@@ -12,6 +12,7 @@
 #include "fused_fwd.cuh"
 #include "fused_fwd_pair.cuh"
 #include "fused_bwd.cuh"
+#include "fused_bwd_pair.cuh"
 
 using namespace qlora;
 
@@ -108,7 +109,8 @@ size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
     return ws_layout(M, N, r, split).total;
 }
 size_t bwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    return ws_layout(M, K, r, plan_gemm(M, K, ceil_div(N, 64)).splits > 1).total;
+    const bool split = !use_pair_fwd(M) && plan_gemm(M, K, ceil_div(N, 64)).splits > 1;
+    return ws_layout(M, K, r, split).total;
 }
 
 // Launches the rank-r tensor-core product out[i*ld_i + j*ld_j] += scaling *
@@ -416,18 +418,52 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
+    // CTA pairs from 64 tokens up (as the forward); the single-CTA kernel with split-K below that
+    const bool pair = use_pair_fwd(M);
     const GemmPlan g = plan_gemm(M, K, ceil_div(N, 64));
-    const WsLayout L = ws_layout(M, K, r, g.splits > 1);
+    const bool split = !pair && g.splits > 1;
+    const WsLayout L = ws_layout(M, K, r, split);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     uint16_t *gs = reinterpret_cast<uint16_t *>(wsb);
     float *gacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
-    float *dxacc = g.splits > 1 ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
+    float *dxacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
     if (r > 0) {
         // G = dY B on tensor cores (B read MN-major), then bf16 copies G and scaling * G
         QL_TRY(cuda_check(cudaMemsetAsync(gacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
         QL_TRY(launch_skinny(dY, 0, B, 1, N, M, r, 1.0f, gacc, r, 1, st));
         QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
     }
+    const Codebook &cb = codebook();
+
+    if (pair) {
+        const int BN = pair_token_tile(M);
+        CUtensorMap tmY, tmC, tmG;
+        QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
+                            CU_TENSOR_MAP_SWIZZLE_64B));
+        if (r > 0)
+            QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
+                                CU_TENSOR_MAP_SWIZZLE_128B));
+        else
+            tmG = tmY;
+        bwdp::Params p;
+        p.scales = w->scales;
+        p.scales2 = w->scales2;
+        p.Alora = A;
+        p.dX = dX;
+        p.M = static_cast<int>(M);
+        p.N = static_cast<int>(N);
+        p.K = static_cast<int>(K);
+        p.r = r;
+        p.BN = BN;
+        for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
+        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel, bwdp::smem_bytes(256)));
+        dim3 grid(static_cast<unsigned>(2 * ceil_div(K, 2 * bwdp::BM)), static_cast<unsigned>(ceil_div(M, BN)), 1);
+        bwdp::fused_bwd_pair_kernel<<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
+        return launch_check("fused_bwd_pair_kernel launch");
+    }
+
     if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
 
     CUtensorMap tmY, tmC, tmG;
@@ -453,7 +489,6 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     p.r = r;
     p.BN = g.BN;
     p.nb_per_split = g.stages_per_split;
-    const Codebook &cb = codebook();
     for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
 
     const int smem = bwd::smem_bytes(g.BN);
