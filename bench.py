@@ -217,6 +217,82 @@ def config_dict(case, n):
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{n}"}
 
 
+# ----------------------------------------------------------------------------- decode sweep
+
+DECODE_LAYERS = 32
+DECODE_MS = (1, 4, 16)
+DECODE_R, DECODE_ALPHA = 8, 16.0
+
+
+def decode_sweep(dev, steps, warmup):
+    """Forward over the 32-layer 7B weight set (Q, K, V, O 4096x4096, up 11008x4096, down
+    4096x11008; LoRA r=8 on Q/K/V/O) at M = 1, 4, 16 tokens, one library call per matrix,
+    captured once in a CUDA graph per M.  Calls carry no data dependency on each other.
+    Returns algorithmic GB/s = (packed weights + X + Y + LoRA A/B bytes) / sweep time."""
+    import torch
+    import bit_quantized_base_nf4_b200 as q
+    from bit_quantized_base_nf4_b200 import synthetic as syn
+    shapes = syn.decode_layer_shapes()
+    r, s = DECODE_R, DECODE_ALPHA / DECODE_R
+    mats = []
+    for layer in range(DECODE_LAYERS):
+        for i, (name, N, K, lora) in enumerate(shapes):
+            w = q.NF4Weight.empty(N, K, device=dev)
+            W = syn.decode_weight(layer, i, N, K, dev)
+            q.qlora_quantize_nf4_dq(W, w)
+            del W
+            A = B = None
+            if lora:
+                A = syn.normal_bf16((r, K), 1.0 / K, 4500 + 16 * layer + i).to(dev)
+                B = syn.normal_bf16((N, r), 0.01, 4700 + 16 * layer + i).to(dev)
+            mats.append((w, N, K, A, B))
+    q.qlora_sync_status()
+    widths = sorted({K for _, _, K, _, _ in mats} | {N for _, N, _, _, _ in mats})
+    out = {}
+    for M in DECODE_MS:
+        X = {K: syn.decode_inputs(M, K, 4900 + K).to(dev) for K in widths}
+        Y = {N: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for N in widths}
+        ws = torch.empty(max(q.qlora_workspace_bytes(M, N, K, r) for _, N, K, _, _ in mats), dtype=torch.uint8,
+                         device=dev)
+        nbytes = 0
+        for w, N, K, A, B in mats:
+            nbytes += q.qlora_packed_bytes(N * K) + 2 * M * K + 2 * M * N
+            if A is not None:
+                nbytes += 2 * r * K + 2 * N * r
+
+        def sweep():
+            for w, N, K, A, B in mats:
+                rr = r if A is not None else 0
+                q.qlora_lora_linear_fwd(w, X[K], A, B, rr, s if rr else 0.0, Y[N], None, ws)
+
+        sweep()                                          # attributes and maps settle outside capture
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            sweep()
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status()
+        ms = a.elapsed_time(b) / steps
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[f"M={M}"] = {"GB/s": gbs, "ms_per_sweep": ms, "bytes_per_sweep": nbytes,
+                         "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
+        del g
+    out["workload"] = ("7B decode sweep: 32 layers x {Q,K,V,O 4096x4096, up 11008x4096, down 4096x11008} = "
+                       f"{sum(N * K for _, N, K, _, _ in mats):.3e} NF4 weights, LoRA r=8 on Q/K/V/O; "
+                       "one forward call per matrix, no inter-call dependency, CUDA graph per M; "
+                       "working set >> L2 (no flush)")
+    out["hbm_peak_gbs"] = peaks()["hbm_gbs"]
+    return out
+
+
 # ----------------------------------------------------------------------------- CUDA leg
 
 def run_ours(args, case):
@@ -318,6 +394,8 @@ def run_ours(args, case):
                 "e2e": {"value": ws * algo_flops(M, N, K, r) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+        if not args.no_decode:
+            line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup)
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(case)
         print(json.dumps(line), flush=True)
@@ -334,6 +412,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-sweep GB/s measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

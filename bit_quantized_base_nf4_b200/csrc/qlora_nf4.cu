@@ -73,10 +73,31 @@ GemmPlan plan_gemm(int64_t M, int64_t rows, int64_t stages) {
     return g;
 }
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current
+// device; the attribute is set once per (kernel, device, size increase), so calls
+// after the first make no CUDA call here.
+struct SmemSetting {
+    const void *kernel;
+    int dev, bytes;
+};
 template <typename K>
 qlora_status set_smem(K kernel, int bytes) {
-    return cuda_check(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
-                      "cudaFuncSetAttribute(max dynamic smem)");
+    static std::mutex mu;
+    static SmemSetting done[256];
+    static int ndone = 0;
+    const void *key = reinterpret_cast<const void *>(kernel);
+    int dev = 0;
+    QL_TRY(cuda_check(cudaGetDevice(&dev), "cudaGetDevice"));
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = -1;
+    for (int i = 0; i < ndone; ++i)
+        if (done[i].kernel == key && done[i].dev == dev) slot = i;
+    if (slot >= 0 && done[slot].bytes >= bytes) return QLORA_OK;
+    QL_TRY(cuda_check(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                      "cudaFuncSetAttribute(max dynamic smem)"));
+    if (slot < 0 && ndone < 256) slot = ndone++;
+    if (slot >= 0) done[slot] = SmemSetting{key, dev, bytes};
+    return QLORA_OK;
 }
 
 qlora_status launch_check(const char *what) { return cuda_check(cudaGetLastError(), what); }

@@ -15,6 +15,11 @@ Workload shapes follow the 7B / 70B layer shapes the source pages quote
 * LoRA A ~ N(0, 1/K) and B ~ N(0, 0.01), rounded to bf16.
 
 N(mu, sigma): the second parameter is the standard deviation.
+
+The 32-layer decode sweep (about 5e9 weights) is the one exception to CPU
+generation: its weights are drawn on the device by torch's CUDA generator,
+seeded per matrix (``decode_weight``), because drawing them on the host would
+take minutes.  A check against the oracle copies the drawn rows to the host.
 """
 from __future__ import annotations
 
@@ -127,3 +132,15 @@ def decode_layer_shapes(with_gate: bool = False) -> list[tuple[str, int, int, bo
     if with_gate:
         shapes.insert(4, ("gate", 11008, 4096, False))
     return shapes
+
+
+def decode_weight(layer: int, index: int, n_out: int, n_in: int, device) -> torch.Tensor:
+    """Weight `index` of decode layer `layer`: N(0, 0.02) fp32 [n_out, n_in] drawn on `device`."""
+    g = torch.Generator(device=device)
+    g.manual_seed(4000 + 16 * int(layer) + int(index))
+    return torch.randn(n_out, n_in, generator=g, dtype=torch.float32, device=device) * 0.02
+
+
+def decode_inputs(M: int, K: int, seed: int) -> torch.Tensor:
+    """Decode activations: M tokens of width K, N(0, 1) rounded to bf16 (host)."""
+    return normal_bf16((M, K), 1.0, seed)
