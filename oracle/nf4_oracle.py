@@ -15,7 +15,7 @@ Pages cited (title, then section):
 * "5.8 QLoRA: 4-bit base + 16-bit sticky notes" (llm-training-guide, qlora)
 * "Training LoRA directly on GGUF quantized weights" (cf-1.com/news/5705389)
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings adopted where the pages are silent:
 
 * NF4 levels: 8 positive and 7 negative normal quantiles with the offset
   delta = ((1 - 1/30) + (1 - 1/32)) / 2, each half divided by
