@@ -13,6 +13,7 @@
 #include "fused_fwd_pair.cuh"
 #include "fused_bwd.cuh"
 #include "fused_bwd_pair.cuh"
+#include "decode_mma.cuh"
 
 using namespace qlora;
 
@@ -125,7 +126,20 @@ int pair_token_tile(int64_t M) {
     const int64_t bn = ceil_div(ceil_div(M, tiles), 32) * 32;
     return static_cast<int>(std::max<int64_t>(32, std::min<int64_t>(256, bn)));
 }
+// Small-M forward: the weight-streaming warp-MMA kernel (decode_mma.cuh), which
+// needs no workspace, for up to 16 tokens and adapter ranks up to 32.
+bool use_decode(int64_t M, int r) { return M <= 16 && r <= dec::kMaxRank; }
+// CTAs per cluster along K: as many as keep every CTA resident (three per SM) and
+// give each warp at least two 64-k blocks; more if the scale table needs it.
+int decode_split(int64_t rowblocks, int64_t KB) {
+    const int64_t cap = 3 * int64_t(sm_count());
+    int S = 1;
+    while (S < 8 && rowblocks * 2 * S <= cap && KB >= int64_t(4) * S * dec::kWarps) S *= 2;
+    while (S < 8 && ceil_div(KB, S) > dec::kMaxBlocks) S *= 2;
+    return S;
+}
 size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    if (use_decode(M, r)) return 0;
     const bool split = !use_pair_fwd(M) && plan_gemm(M, N, K / 64).splits > 1;
     return ws_layout(M, N, r, split).total;
 }
@@ -323,6 +337,60 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     QL_TRY(check_ws(ws, ws_bytes, need));
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (use_decode(M, r)) {
+        const int64_t KB = K / 64, rowblocks = ceil_div(N, dec::kRows);
+        const int S = decode_split(rowblocks, KB);
+        if (ceil_div(KB, S) > dec::kMaxBlocks)
+            return fail(QLORA_ERR_SHAPE, "n_in (%lld) too large for the small-M path", (long long)K);
+        dec::Params p;
+        p.codes = w->codes;
+        p.scales = w->scales;
+        p.scales2 = w->scales2;
+        p.X = X;
+        p.Alora = r > 0 ? A : nullptr;
+        p.Blora = r > 0 ? B : nullptr;
+        p.Y = Y;
+        p.U_save = r > 0 ? U_save : nullptr;
+        p.M = static_cast<int>(M);
+        p.N = static_cast<int>(N);
+        p.K = static_cast<int>(K);
+        p.r = r;
+        p.S = S;
+        p.blocks_per_cta = static_cast<int>(ceil_div(KB, S));
+        p.scaling = scaling;
+        const Codebook &cbd = codebook();
+        for (int i = 0; i < 16; ++i) p.level[i] = cbd.level[i];
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(rowblocks * S));
+        cfg.blockDim = dim3(dec::kThreads);
+        cfg.dynamicSmemBytes = dec::smem_bytes();
+        cfg.stream = st;
+        cudaLaunchAttribute at[2];
+        int na = 0;
+        // programmatic dependent launch: the kernel prefetches its frozen weights into L2
+        // before waiting for the preceding grid
+        at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+        if (S > 1) {
+            at[na].id = cudaLaunchAttributeClusterDimension;
+            at[na].val.clusterDim.x = static_cast<unsigned>(S);
+            at[na].val.clusterDim.y = 1;
+            at[na].val.clusterDim.z = 1;
+            ++na;
+        }
+        cfg.attrs = at;
+        cfg.numAttrs = na;
+        if (M <= 8) {
+            QL_TRY(set_smem(dec::decode_kernel<1>, dec::smem_bytes()));
+            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<1>, p), "decode_kernel launch"));
+        } else {
+            QL_TRY(set_smem(dec::decode_kernel<2>, dec::smem_bytes()));
+            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<2>, p), "decode_kernel launch"));
+        }
+        return QLORA_OK;
+    }
 
     const bool pair = use_pair_fwd(M);
     const GemmPlan g = plan_gemm(M, N, K / 64);

@@ -87,10 +87,11 @@ def test_validation_rejects_before_launch(lib):
     assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 0, A, B, 8, 2.0, Y, None, ws, 1 << 20, None) == 2
     assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 16, A, B, 8, float("nan"), Y, None, ws, 1 << 20,
                                      None) == 1
-    # workspace too small / missing
-    assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 16, A, B, 8, 2.0, Y, None, ws, 8, None) == 4
-    assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 16, A, B, 8, 2.0, Y, None, None, 0, None) == 4
-    assert lib.qlora_lora_linear_bwd_dx(ctypes.byref(w), X, 16, A, B, 8, 2.0, Y, None, ws, 8, None) == 4
+    # workspace too small / missing (64 tokens: the adapter's rank buffers live in the workspace)
+    assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 64, A, B, 8, 2.0, Y, None, ws, 8, None) == 4
+    assert lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 64, A, B, 8, 2.0, Y, None, None, 0, None) == 4
+    assert lib.qlora_lora_linear_bwd_dx(ctypes.byref(w), X, 64, A, B, 8, 2.0, Y, None, ws, 8, None) == 4
+
     # misaligned activations
     assert lib.qlora_lora_linear_fwd(ctypes.byref(w), ctypes.c_void_p(0x10002), 16, A, B, 8, 2.0, Y, None, ws,
                                      1 << 20, None) == 3

@@ -122,6 +122,16 @@ CASES = [
     syn.LayerCase("decode-m1-n4096-k4096-r8", M=1, N=4096, K=4096, r=8, alpha=16.0, seed=105),
     syn.LayerCase("decode-m4-n1024-k11008-r8", M=4, N=1024, K=11008, r=8, alpha=16.0, seed=106),
     syn.LayerCase("decode-m16-n2048-k4096-r8", M=16, N=2048, K=4096, r=8, alpha=16.0, seed=107),
+    # small-M kernel edges: 12 tokens (second token tile partly empty), ragged rows, one CTA per cluster
+    syn.LayerCase("decode-m12-n200-k704-r16", M=12, N=200, K=704, r=16, alpha=32.0, seed=109),
+    # largest fused adapter rank, four-CTA clusters
+    syn.LayerCase("decode-m1-n4096-k4096-r32", M=1, N=4096, K=4096, r=32, alpha=64.0, seed=110),
+    # the 7B down projection at full size, 16 tokens, base only
+    syn.LayerCase("decode-m16-n4096-k11008-r0", M=16, N=4096, K=11008, r=0, alpha=0.0, seed=111),
+    # adapter rank above the small-M kernel's limit: split-K tensor-core path
+    syn.LayerCase("small-m8-n256-k1024-r64", M=8, N=256, K=1024, r=64, alpha=128.0, seed=112),
+    # between the small-M kernel and the CTA-pair kernels: split-K tensor-core path
+    syn.LayerCase("small-m40-n384-k2048-r8", M=40, N=384, K=2048, r=8, alpha=16.0, seed=113),
     syn.LayerCase("m600-n512-k768-r8-2tiles", M=600, N=512, K=768, r=8, alpha=16.0, seed=108),
 ]
 

@@ -20,8 +20,10 @@ DEV = "cuda"
 CASES = [
     # CTA-pair forward (M >= 64), ragged in every dimension
     syn.LayerCase("pair-m300-n320-k576-r16", M=300, N=320, K=576, r=16, alpha=32.0, seed=201),
-    # decode shape: single-CTA forward with a split-K accumulator in the scratch
-    syn.LayerCase("split-m4-n512-k2048-r8", M=4, N=512, K=2048, r=8, alpha=16.0, seed=202),
+    # 32 tokens: single-CTA forward with a split-K accumulator in the scratch
+    syn.LayerCase("split-m32-n512-k2048-r8", M=32, N=512, K=2048, r=8, alpha=16.0, seed=202),
+    # 4 tokens: the small-M kernel, which needs no scratch
+    syn.LayerCase("decode-m4-n512-k2048-r8", M=4, N=512, K=2048, r=8, alpha=16.0, seed=205),
     # no adapter
     syn.LayerCase("base-only-m64-n256-k512", M=64, N=256, K=512, r=0, alpha=0.0, seed=203),
     # 7B attention projection at 2048 tokens, rank 8
