@@ -29,6 +29,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fused NF4-dequant LoRA linear TFLOP/s (fwd+bwd)"
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kernel on this
+# workload, from one ncu capture each (profiles/); set to None when the kernel changes
+KERNEL_TRAFFIC = {"dx": 25_607_680, "fwd": 25_583_104}
 UNIT = "TFLOP/s"
 
 
@@ -224,7 +228,7 @@ DECODE_MS = (1, 4, 16)
 DECODE_R, DECODE_ALPHA = 8, 16.0
 
 
-def decode_sweep(dev, steps, warmup):
+def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS):
     """Forward over the 32-layer 7B weight set (Q, K, V, O 4096x4096, up 11008x4096, down
     4096x11008; LoRA r=8 on Q/K/V/O) at M = 1, 4, 16 tokens, one library call per matrix,
     captured once in a CUDA graph per M.  Calls carry no data dependency on each other.
@@ -235,7 +239,7 @@ def decode_sweep(dev, steps, warmup):
     shapes = syn.decode_layer_shapes()
     r, s = DECODE_R, DECODE_ALPHA / DECODE_R
     mats = []
-    for layer in range(DECODE_LAYERS):
+    for layer in range(layers):
         for i, (name, N, K, lora) in enumerate(shapes):
             w = q.NF4Weight.empty(N, K, device=dev)
             W = syn.decode_weight(layer, i, N, K, dev)
@@ -285,7 +289,7 @@ def decode_sweep(dev, steps, warmup):
         out[f"M={M}"] = {"GB/s": gbs, "ms_per_sweep": ms, "bytes_per_sweep": nbytes,
                          "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
         del g
-    out["workload"] = ("7B decode sweep: 32 layers x {Q,K,V,O 4096x4096, up 11008x4096, down 4096x11008} = "
+    out["workload"] = (f"7B decode sweep: {layers} layers x {{Q,K,V,O 4096x4096, up 11008x4096, down 4096x11008}} = "
                        f"{sum(N * K for _, N, K, _, _ in mats):.3e} NF4 weights, LoRA r=8 on Q/K/V/O; "
                        "one forward call per matrix, no inter-call dependency, CUDA graph per M; "
                        "working set >> L2 (no flush)")
@@ -375,27 +379,56 @@ def run_ours(args, case):
     h2d = (hX.numel() + hdY.numel()) * 2
     d2h = (hdA.numel() + hdB.numel()) * 4
 
+    # the two GEMM kernels alone: with r = 0 each call is exactly one launch of the fused
+    # kernel (dX: CTA-pair transposed-dequant GEMM; forward: CTA-pair dequant GEMM)
+    kern = {"dx": [], "fwd": []}
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        q.qlora_lora_linear_bwd_dx(w, dY, None, None, 0, 0.0, dX, None, wsb, stream=stream)
+        b.record(stream)
+        flush.fill_((i + 1) & 0xFF)
+        b2 = torch.cuda.Event(enable_timing=True)
+        b2.record(stream)
+        q.qlora_lora_linear_fwd(w, X, None, None, 0, 0.0, Y, None, wsb, stream=stream)
+        c.record(stream)
+        if i >= args.warmup:
+            kern["dx"].append((a, b))
+            kern["fwd"].append((b2, c))
+    torch.cuda.synchronize(dev)
+    q.qlora_sync_status(stream)
+    dx_k_ms = statistics.mean(x.elapsed_time(y) for x, y in kern["dx"])
+    fwd_k_ms = statistics.mean(x.elapsed_time(y) for x, y in kern["fwd"])
+    base_flops = 2 * M * N * K
+
     pk = peaks()
-    fwd_avg = statistics.mean(fwd_ms)
-    achieved = fwd_flops(M, N, K, r) / (fwd_avg * 1e-3) / 1e12
-    roof = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": achieved / pk["bf16_tflops"], "traffic": None,
-            "kernel": "forward call (fused NF4-dequant tcgen05 GEMM + its X A^T side kernel)",
-            "peak_source": f"{pk['source']} bf16 burst", "frac_of_sustained":
-                (achieved / pk["bf16_tflops_sustained"]) if pk.get("bf16_tflops_sustained") else None}
+
+    def roofline(ms, name, traffic):
+        achieved = base_flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / pk["bf16_tflops"], "traffic": traffic, "kernel": name,
+                "launch_ms": ms, "flops_per_launch": base_flops,
+                "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json)",
+                "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"])
+                if pk.get("bf16_tflops_sustained") else None}
+
+    # dram bytes per launch from ncu captures of this workload (see profiles/), None once stale
+    roof = roofline(dx_k_ms, "fused_bwd_pair_kernel (dX, dominant kernel of the step)", KERNEL_TRAFFIC.get("dx"))
+    roof_fwd = roofline(fwd_k_ms, "fused_fwd_pair_kernel (forward base GEMM)", KERNEL_TRAFFIC.get("fwd"))
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(case, ws),
-                "roofline": roof,
+                "roofline": roof, "roofline_fwd": roof_fwd,
                 "phases_ms": {"fwd": statistics.mean(fwd_ms), "bwd_dx": statistics.mean(dx_ms),
                               "grad_ab": statistics.mean(grad_ms)},
                 "e2e": {"value": ws * algo_flops(M, N, K, r) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         if not args.no_decode:
-            line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup)
+            line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers)
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(case)
         print(json.dumps(line), flush=True)
@@ -413,6 +446,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-sweep GB/s measurement")
+    ap.add_argument("--decode-only", action="store_true", help="run only the decode sweep (prints its JSON)")
+    ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -420,6 +455,11 @@ def main():
     case = syn.attn7b_case()
     if args.impl == "reference":
         run_reference(args, case)
+    elif args.decode_only:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"decode": decode_sweep(dev, args.steps, args.warmup, args.decode_layers)}), flush=True)
     else:
         run_ours(args, case)
 

@@ -18,7 +18,7 @@
 //
 // Work split.  A CTA (4 warps) owns 64 W rows and a contiguous range of 64-k blocks;
 // the S CTAs of a cluster cover all of K for the same rows (S = 1, 2, 4 or 8).
-// Warps take the CTA's blocks round-robin and accumulate all 64 rows.  Partial sums
+// Each warp takes a contiguous quarter of the CTA's blocks and accumulates all 64 rows.  Partial sums
 // are added across warps in shared memory and across the cluster through
 // distributed shared memory by the cluster's first CTA, which also adds the
 // adapter term and writes Y.  U is computed by the same loop: the rows of A are a
@@ -96,9 +96,11 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
                  : "l"(p));
     return v;
 }
+// 8 bytes of a code row; a miss fetches the whole 256-byte aligned span into L2, which
+// holds the warp's next blocks of the same row
 __device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
     uint2 v;
-    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    asm volatile("ld.global.nc.L2::256B.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;
 }
 
@@ -182,9 +184,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
     float dn[kGroups];
     uint4 xn[4];
     uint4 an[kMaxRank / 8][2];
-    int kb = kb0 + warp;
+    // warp w takes a contiguous run of the CTA's blocks
+    const int per_warp = (nbc + kWarps - 1) / kWarps;
+    const int wk0 = kb0 + warp * per_warp, wk1 = min(kb1, wk0 + per_warp);
+    int kb = wk0;
     auto load_block = [&](int k) {
-        const bool in = k < kb1;
+        const bool in = k < wk1;
 #pragma unroll
         for (int grp = 0; grp < kGroups; ++grp) {
             const bool v = in && rvalid[grp];
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
     };
     load_block(kb);
 
-    for (; kb < kb1; kb += kWarps) {
+    for (; kb < wk1; ++kb) {
         uint2 ccur[kGroups];
         uint32_t s2c[kGroups];
 #pragma unroll
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const Params p) {
             aw[u][0] = an[u][0].x; aw[u][1] = an[u][0].y; aw[u][2] = an[u][0].z; aw[u][3] = an[u][0].w;
             aw[u][4] = an[u][1].x; aw[u][5] = an[u][1].y; aw[u][6] = an[u][1].z; aw[u][7] = an[u][1].w;
         }
-        load_block(kb + kWarps);
+        load_block(kb + 1);
 
 #pragma unroll
         for (int grp = 0; grp < kGroups; ++grp) {
