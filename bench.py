@@ -297,6 +297,35 @@ def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS):
     return out
 
 
+# ----------------------------------------------------------------------------- quantize pass
+
+def quantize_pass(dev, steps, warmup):
+    """One-shot encode (NF4 codes + double-quantized scales) of the 70B FFN up projection,
+    28672 x 8192 fp32 ~N(0, 0.015) drawn on the device; GB/s = (4 + packed bytes per weight)
+    x weights / time.  The 0.94 GB input is far larger than L2."""
+    import torch
+    import bit_quantized_base_nf4_b200 as q
+    N, K = 28672, 8192
+    g = torch.Generator(device=dev)
+    g.manual_seed(5100)
+    W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32) * 0.015
+    w = q.NF4Weight.empty(N, K, device=dev)
+    for _ in range(warmup):
+        q.qlora_quantize_nf4_dq(W, w)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        q.qlora_quantize_nf4_dq(W, w)
+    b.record()
+    torch.cuda.synchronize(dev)
+    q.qlora_sync_status()
+    ms = a.elapsed_time(b) / steps
+    nbytes = 4 * N * K + q.qlora_packed_bytes(N * K)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "70B FFN up 28672x8192 fp32 -> NF4 + DQ", "ms": ms, "bytes": nbytes, "GB/s": gbs,
+            "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
+
+
 # ----------------------------------------------------------------------------- CUDA leg
 
 def run_ours(args, case):
@@ -428,6 +457,7 @@ def run_ours(args, case):
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         if not args.no_decode:
+            line["quantize"] = quantize_pass(dev, max(5, args.steps // 2), args.warmup)
             line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers)
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(case)

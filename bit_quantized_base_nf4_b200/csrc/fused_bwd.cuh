@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idesc = make_idesc_bf16(BM, p.BN, 1, 0);
+            int done = 0;
             for (int s = 0; s < total; ++s) {
                 const int sx = s % SX, sa = s % SA;
                 if (!mbar_wait(&y_full[sx], (s / SX) & 1, abort_flag)) break;
@@ -161,9 +162,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_commit(&y_empty[sx]);
                 tc_commit(&a_empty[sa]);
+                done = s + 1;
             }
             tc_commit(acc_full);
             mbar_drain(acc_full, 0);
+            // every release commit has landed before the CTA exits, so none can reach the
+            // shared memory of a CTA launched after it
+            for (int s = max(0, done - SX); s < done; ++s) mbar_drain(&y_empty[s % SX], (s / SX) & 1);
+            for (int s = max(0, done - SA); s < done; ++s) mbar_drain(&a_empty[s % SA], (s / SA) & 1);
         }
     } else if (warp >= 4) {
         // thread = (contraction row nl, k half h): one 64-block of W0 row n

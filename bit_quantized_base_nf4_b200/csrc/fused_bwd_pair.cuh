@@ -138,7 +138,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int s = 0; s < total; ++s) {
                 const int sx = s % S;
-                if (!mbar_wait(&free_b[sx], ((s / S) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait_cluster(&free_b[sx], ((s / S) & 1) ^ 1, abort_flag)) break;
                 const uint32_t bar0 = mapa_shared(smem_u32(&y_full[sx]), 0);
                 if (rank == 0) mbar_arrive_expect_tx(&y_full[sx], 2 * ysb);
                 if (s < NB)
@@ -150,6 +150,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // the even CTA sees both CTAs' copies complete on its barriers
             if (rank == 0)
                 for (int s = max(0, issued - S); s < issued; ++s) mbar_drain(&y_full[s % S], (s / S) & 1);
+            // producer tail: the release commits of the last stages land on this CTA's barriers
+            // before it exits, so none can reach the shared memory of a CTA launched after it
+            for (int s = max(0, issued - S); s < issued; ++s) mbar_drain_cluster(&free_b[s % S], (s / S) & 1);
         }
     } else if (warp == 3) {
         // ---------------- packed-code producer (local to each CTA)
@@ -259,7 +262,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
             // A slot g is free once the MMAs of stage s - 4 have completed
-            if (!mbar_wait(&free_b[g], ((s / S) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_cluster(&free_b[g], ((s / S) & 1) ^ 1, abort_flag)) { ok = false; break; }
             const uint32_t abase = sAu + g * kAStageBytes + a_off;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -269,13 +272,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             // the even CTA's warps arrive only once the stage's dY tile (both halves) has landed,
             // so a completed a_full also means a completed y_full for the MMA thread
-            if (rank == 0 && !mbar_wait(&y_full[g], (s / S) & 1, abort_flag)) { ok = false; break; }
+            if (rank == 0 && !mbar_wait_cluster(&y_full[g], (s / S) & 1, abort_flag)) { ok = false; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
         }
 
         // ---------------- epilogue: this CTA's 128 k rows x BN tokens
-        if (ok && mbar_wait(acc_full, 0, abort_flag)) {
+        if (ok && mbar_wait_cluster(acc_full, 0, abort_flag)) {
             tc_fence_after();
             const int quad = warp & 3;
             const int row = quad * 32 + lane;

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc = make_idesc_bf16(BM, p.BN, 0, 0);
+            int done = 0;
             for (int s = 0; s < total; ++s) {
                 const int sx = s % SX, sa = s % SA;
                 if (!mbar_wait(&x_full[sx], (s / SX) & 1, abort_flag)) break;
@@ -173,10 +174,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_commit(&x_empty[sx]);
                 tc_commit(&a_empty[sa]);
+                done = s + 1;
             }
             tc_commit(acc_full);
             // the accumulator (and TMEM) must not be released while MMAs are in flight
             mbar_drain(acc_full, 0);
+            // every release commit has landed before the CTA exits, so none can reach the
+            // shared memory of a CTA launched after it
+            for (int s = max(0, done - SX); s < done; ++s) mbar_drain(&x_empty[s % SX], (s / SX) & 1);
+            for (int s = max(0, done - SA); s < done; ++s) mbar_drain(&a_empty[s % SA], (s / SA) & 1);
         }
     } else if (warp >= 4) {
         // ---------------- dequant into TMEM, then epilogue
@@ -247,8 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!mbar_wait(&a_empty[sa], ((s / SA) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            tmem_st32(tmem_a + lane_addr + sa * 32, out);
-            tmem_wait_st();
+            tmem_st32_checked(tmem_a + lane_addr + sa * 32, out);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[sa]);

@@ -132,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int q = 0; q < Q; ++q) {
                 const int sx = q % SX;
-                if (!mbar_wait(&free_b[sx], ((q / SX) & 1) ^ 1, abort_flag)) break;
+                if (!mbar_wait_cluster(&free_b[sx], ((q / SX) & 1) ^ 1, abort_flag)) break;
                 const uint32_t bar0 = mapa_shared(smem_u32(&x_full[sx]), 0);
                 uint8_t *slot = sX + sx * slotb;
                 if (q < QM) {
@@ -148,6 +148,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // the even CTA sees both CTAs' copies complete on its barriers
             if (rank == 0)
                 for (int q = max(0, issued - SX); q < issued; ++q) mbar_drain(&x_full[q % SX], (q / SX) & 1);
+            // producer tail: the release commits of the last stages land on this CTA's barriers
+            // before it exits, so none can reach the shared memory of a CTA launched after it
+            for (int q = max(0, issued - SX); q < issued; ++q) mbar_drain_cluster(&free_b[q % SX], (q / SX) & 1);
         }
     } else if (warp == 3) {
         // ---------------- packed-code producer (local to each CTA)
@@ -169,7 +172,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t idesc = make_idesc_bf16(2 * BM, p.BN, 0, 0);
             for (int q = 0; q < Q; ++q) {
                 const int sx = q % SX, g = q % kGroups;
-                if (!mbar_wait(&a_full[g], (q / kGroups) & 1, abort_flag)) break;
+                // the peer CTA's half of the A operand was written by its threads: acquire at cluster scope
+                if (!mbar_wait_cluster(&a_full[g], (q / kGroups) & 1, abort_flag)) break;
                 tc_fence_after();
                 // MMAs of this stage: 8 for a full main stage, 4 for the last odd chunk,
                 // ceil(r/16) for the adapter stage
@@ -218,7 +222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
         for (int q = grp; q < Q && ok; q += kGroups) {
             const int g = grp;
-            if (!mbar_wait(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_cluster(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             if (q < QM) {
                 const int ci = q >> 1, sc = ci % SC;
@@ -252,7 +256,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
                         }
                     }
-                    tmem_st32(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
                 }
             } else {
                 // adapter stage: A operand = B_lora row n, elements 0 .. 127 (zero past r)
@@ -268,20 +272,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             w = __ldg(reinterpret_cast<const uint4 *>(p.Blora + int64_t(n) * p.r + e0));
                         out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
                     }
-                    tmem_st32(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
                 }
             }
-            tmem_wait_st();
             tc_fence_before();
             // the even CTA's warps arrive only once the stage's X tile (both halves) has landed,
             // so a completed a_full also means a completed x_full for the MMA thread
-            if (rank == 0 && !mbar_wait(&x_full[g], (q / kGroups) & 1, abort_flag)) { ok = false; break; }
+            if (rank == 0 && !mbar_wait_cluster(&x_full[g], (q / kGroups) & 1, abort_flag)) { ok = false; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
         }
 
         // ---------------- epilogue: this CTA's 128 rows x BN tokens
-        if (ok && mbar_wait(acc_full, 0, abort_flag)) {
+        if (ok && mbar_wait_cluster(acc_full, 0, abort_flag)) {
             tc_fence_after();
             const int nchunks = p.BN / 16;
             for (int ch = grp; ch < nchunks; ch += kGroups) {

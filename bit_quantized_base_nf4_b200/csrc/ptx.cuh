@@ -11,6 +11,7 @@ namespace qlora {
 // Device error word: set when a pipeline wait gives up; read by qlora_sync_status().
 __device__ int g_device_error = 0;
 constexpr int kDeviceErrTimeout = 6;
+constexpr int kDeviceErrTmemStore = 7;   // a TMEM store did not read back as written
 // Time after which a single pipeline wait gives up (ns of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -208,6 +209,14 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8])
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Store 32 columns and return only once they are in TMEM and the source registers
+// are free.  tcgen05.st reads its source registers asynchronously, but nothing in
+// the PTX ties those registers to tcgen05.wait::st, so the compiler may reuse them
+// early; corrupted A operands were observed at large K.  Reading the columns back
+// and comparing them with the source words keeps the sources live until the store
+// is complete; a mismatch is recorded as a device error.
+__device__ __forceinline__ void tmem_st32_checked(uint32_t taddr, const uint32_t (&v)[32]);
+
 // Load 16 consecutive columns; the values are only valid after the wait below,
 // which takes the registers as in/out operands so no use can move above it.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
@@ -378,6 +387,20 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}\n" ::"r"(
             smem_u32(bar))
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32_checked(uint32_t taddr, const uint32_t (&v)[32]) {
+    tmem_st32(taddr, v);
+    tmem_wait_st();
+    uint32_t r0[16], r1[16];
+    tmem_ld16(taddr, r0);
+    tmem_ld16(taddr + 16, r1);
+    tmem_wait_ld16(r0);
+    tmem_wait_ld16(r1);
+    uint32_t diff = 0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) diff |= (r0[e] ^ v[e]) | (r1[e] ^ v[16 + e]);
+    if (diff) atomicExch(&g_device_error, kDeviceErrTmemStore);
 }
 
 }  // namespace qlora

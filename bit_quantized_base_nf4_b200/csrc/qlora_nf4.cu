@@ -286,6 +286,8 @@ qlora_status qlora_sync_status(void *stream) {
     if (v) {
         const int zero = 0;
         cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+        if (v == kDeviceErrTmemStore)
+            return fail(QLORA_ERR_CUDA, "a tensor-memory store did not read back as written (device error %d)", v);
         return fail(QLORA_ERR_TIMEOUT, "a kernel pipeline wait timed out (device error %d)", v);
     }
     return QLORA_OK;

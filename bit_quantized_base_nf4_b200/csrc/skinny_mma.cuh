@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0 && nu > 0) {
             const uint32_t idesc = make_idesc_bf16(BI, p.Nq, p.p_mn, p.q_mn);
-            int seg = 0;
+            int seg = 0, done = 0;
             for (int k = 0; k < nu; ++k) {
                 const int64_t u = u_begin + k;
                 const bool first = (k == 0) || (u % ST == 0);
@@ -171,10 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_commit(&acc_full[buf]);
                     ++seg;
                 }
+                done = k + 1;
             }
             // TMEM is released only after every MMA has completed
             tc_commit(mma_done);
             mbar_drain(mma_done, 0);
+            // every release commit has landed before the CTA exits, so none can reach the
+            // shared memory of a CTA launched after it
+            for (int k = max(0, done - S); k < done; ++k) mbar_drain(&empty[k % S], (k / S) & 1);
         }
     } else if (nu > 0) {
         // epilogue, warps 2-5: TMEM lane quadrant (warp % 4), one output row i per thread

@@ -177,8 +177,10 @@ qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const
                                 const qlora_bf16 *G, int64_t M, int64_t N, int64_t K, int r,
                                 float scaling, float *dA, float *dB, int accumulate, void *stream);
 
-/* Waits for `stream`, then reports and clears a device-side timeout
- * recorded by any earlier kernel of this library on the current device. */
+/* Waits for `stream`, then reports and clears a device-side error recorded by
+ * any earlier kernel of this library on the current device: a pipeline wait
+ * that timed out (QLORA_ERR_TIMEOUT) or a tensor-memory store whose read-back
+ * check failed (QLORA_ERR_CUDA). */
 qlora_status qlora_sync_status(void *stream);
 
 /* Message describing the last failure on the calling thread ("" if none). */
