@@ -212,9 +212,10 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // Store 32 columns and return only once they are in TMEM and the source registers
 // are free.  tcgen05.st reads its source registers asynchronously, but nothing in
 // the PTX ties those registers to tcgen05.wait::st, so the compiler may reuse them
-// early; corrupted A operands were observed at large K.  Reading the columns back
-// and comparing them with the source words keeps the sources live until the store
-// is complete; a mismatch is recorded as a device error.
+// early; corrupted A operands were observed at large K.  Reading every stored
+// column back and comparing it with its source word keeps the sources live until
+// the store is complete (a read-back of one column alone did not suffice); a
+// mismatch is recorded as a device error.
 __device__ __forceinline__ void tmem_st32_checked(uint32_t taddr, const uint32_t (&v)[32]);
 
 // Load 16 consecutive columns; the values are only valid after the wait below,
