@@ -32,7 +32,7 @@ METRIC = "fused NF4-dequant LoRA linear TFLOP/s (fwd+bwd)"
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kernel on this
 # workload, from one ncu capture each (profiles/); set to None when the kernel changes
-KERNEL_TRAFFIC = {"dx": None, "fwd": None}
+KERNEL_TRAFFIC = {"dx": 25_606_400, "fwd": 25_710_592}
 UNIT = "TFLOP/s"
 
 
