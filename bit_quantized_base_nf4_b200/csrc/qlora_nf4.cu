@@ -127,19 +127,49 @@ int pair_token_tile(int64_t M) {
     return static_cast<int>(std::max<int64_t>(32, std::min<int64_t>(256, bn)));
 }
 // Small-M forward: the weight-streaming warp-MMA kernel (decode_mma.cuh), which
-// needs no workspace, for up to 16 tokens and adapter ranks up to 32.
-bool use_decode(int64_t M, int r) { return M <= 16 && r <= dec::kMaxRank; }
-// CTAs per cluster along K: as many as keep every CTA resident (three per SM) and
-// give each warp at least two 64-k blocks; more if the scale table needs it.
-int decode_split(int64_t rowblocks, int64_t KB) {
-    const int64_t cap = 3 * int64_t(sm_count());
-    int S = 1;
-    while (S < 8 && rowblocks * 2 * S <= cap && KB >= int64_t(4) * S * dec::kWarps) S *= 2;
-    while (S < 8 && ceil_div(KB, S) > dec::kMaxBlocks) S *= 2;
-    return S;
+// needs no workspace, for up to 16 tokens, adapter ranks up to 16 and n_in up to 32768.
+bool use_decode(int64_t M, int64_t K, int r) { return M <= 16 && r <= dec::kMaxRank && K / 64 <= dec::kMaxKB; }
+
+// Shared-memory plan of the small-M kernel: table, code ring, activation ring, two
+// scale buffers, partial sums, barriers.  The rings are as deep as the 227 KB allow.
+struct DecodePlan {
+    dec::Params p;
+    int smem;
+};
+DecodePlan plan_decode(int64_t M, int64_t K, int r) {
+    DecodePlan d{};
+    dec::Params &p = d.p;
+    const int KB = static_cast<int>(K / 64);
+    p.mbox = M <= 8 ? 8 : 16;
+    p.rbox = r == 0 ? 0 : (r <= 8 ? 8 : 16);
+    const int sc_q = (dec::kRows * KB + 16 + 15) & ~15;
+    const int s2_floats = ((dec::kRows * KB) / 256 + 2 + 3) & ~3;
+    p.sc_q = sc_q;
+    p.sc_stage = (sc_q + 4 * s2_floats + 127) & ~127;
+    p.xa_stage = (p.mbox + p.rbox) * 1024;
+    auto total = [&](int dc, int dx) {
+        p.dc = dc;
+        p.dx = dx;
+        p.off_code = dec::kLutBytes;
+        p.off_xa = p.off_code + dc * dec::kCodeStage;
+        p.off_sc = p.off_xa + dx * p.xa_stage;
+        p.off_part = p.off_sc + 2 * p.sc_stage;
+        p.off_upart = p.off_part + 2 * dec::kPartFloats * 4;
+        p.off_ufin = p.off_upart + 4 * 256 * 4;
+        p.off_bars = p.off_ufin + 256 * 4;
+        const int bars = (2 * dec::kMaxCodeStages + 2 * dec::kMaxXaStages + 4) * 8 + 16;
+        return 1024 + p.off_bars + bars;   // + alignment slack of the dynamic base
+    };
+    int dc = dec::kMaxCodeStages, dx = dec::kMaxXaStages;
+    while (total(dc, dx) > dec::kSmemLimit && (dx > 2 || dc > 4)) {
+        if (dx > 2) --dx;
+        else --dc;
+    }
+    d.smem = total(dc, dx);
+    return d;
 }
 size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    if (use_decode(M, r)) return 0;
+    if (use_decode(M, K, r)) return 0;
     const bool split = !use_pair_fwd(M) && plan_gemm(M, N, K / 64).splits > 1;
     return ws_layout(M, N, r, split).total;
 }
@@ -340,17 +370,14 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    if (use_decode(M, r)) {
-        const int64_t KB = K / 64, rowblocks = ceil_div(N, dec::kRows);
-        const int S = decode_split(rowblocks, KB);
-        if (ceil_div(KB, S) > dec::kMaxBlocks)
+    if (use_decode(M, K, r)) {
+        DecodePlan d = plan_decode(M, K, r);
+        if (d.smem > dec::kSmemLimit)
             return fail(QLORA_ERR_SHAPE, "n_in (%lld) too large for the small-M path", (long long)K);
-        dec::Params p;
+        dec::Params &p = d.p;
         p.codes = w->codes;
         p.scales = w->scales;
         p.scales2 = w->scales2;
-        p.X = X;
-        p.Alora = r > 0 ? A : nullptr;
         p.Blora = r > 0 ? B : nullptr;
         p.Y = Y;
         p.U_save = r > 0 ? U_save : nullptr;
@@ -358,38 +385,35 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         p.N = static_cast<int>(N);
         p.K = static_cast<int>(K);
         p.r = r;
-        p.S = S;
-        p.blocks_per_cta = static_cast<int>(ceil_div(KB, S));
+        p.units = static_cast<int>(ceil_div(N, dec::kRows));
         p.scaling = scaling;
         const Codebook &cbd = codebook();
         for (int i = 0; i < 16; ++i) p.level[i] = cbd.level[i];
+        // codes as u8 [N, K/2]: [32 rows x 128 B] boxes; X and A as [K/64][rows][64] bf16 chunks
+        CUtensorMap tmC, tmX, tmA;
+        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, dec::kRows, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(make_tmap_chunks(&tmX, X, M, K, p.mbox, dec::kStageBlocks));
+        if (r > 0) QL_TRY(make_tmap_chunks(&tmA, A, r, K, p.rbox, dec::kStageBlocks));
+        else tmA = tmX;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(rowblocks * S));
+        cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(p.units, sm_count())));
         cfg.blockDim = dim3(dec::kThreads);
-        cfg.dynamicSmemBytes = dec::smem_bytes();
+        cfg.dynamicSmemBytes = d.smem;
         cfg.stream = st;
-        cudaLaunchAttribute at[2];
-        int na = 0;
-        // programmatic dependent launch: the kernel prefetches its frozen weights into L2
-        // before waiting for the preceding grid
-        at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        at[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-        if (S > 1) {
-            at[na].id = cudaLaunchAttributeClusterDimension;
-            at[na].val.clusterDim.x = static_cast<unsigned>(S);
-            at[na].val.clusterDim.y = 1;
-            at[na].val.clusterDim.z = 1;
-            ++na;
-        }
+        // programmatic dependent launch: the kernel builds its table and warms L2 with its
+        // frozen weights before waiting for the preceding grid
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
-        cfg.numAttrs = na;
+        cfg.numAttrs = 1;
         if (M <= 8) {
-            QL_TRY(set_smem(dec::decode_kernel<1>, dec::smem_bytes()));
-            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<1>, p), "decode_kernel launch"));
+            QL_TRY(set_smem(dec::decode_kernel<1>, d.smem));
+            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<1>, tmC, tmX, tmA, p), "decode_kernel launch"));
         } else {
-            QL_TRY(set_smem(dec::decode_kernel<2>, dec::smem_bytes()));
-            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<2>, p), "decode_kernel launch"));
+            QL_TRY(set_smem(dec::decode_kernel<2>, d.smem));
+            QL_TRY(cuda_check(cudaLaunchKernelEx(&cfg, dec::decode_kernel<2>, tmC, tmX, tmA, p), "decode_kernel launch"));
         }
         return QLORA_OK;
     }

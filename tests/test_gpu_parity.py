@@ -122,9 +122,20 @@ CASES = [
     syn.LayerCase("decode-m1-n4096-k4096-r8", M=1, N=4096, K=4096, r=8, alpha=16.0, seed=105),
     syn.LayerCase("decode-m4-n1024-k11008-r8", M=4, N=1024, K=11008, r=8, alpha=16.0, seed=106),
     syn.LayerCase("decode-m16-n2048-k4096-r8", M=16, N=2048, K=4096, r=8, alpha=16.0, seed=107),
-    # small-M kernel edges: 12 tokens (second token tile partly empty), ragged rows, one CTA per cluster
+    # small-M kernel edges: 12 tokens (second token tile partly empty), ragged last unit
+    # (200 = 6 x 32 + 8 rows) and ragged last stage (11 of 16 blocks)
     syn.LayerCase("decode-m12-n200-k704-r16", M=12, N=200, K=704, r=16, alpha=32.0, seed=109),
-    # largest fused adapter rank, four-CTA clusters
+    # one unit of 8 rows, one 64-k block
+    syn.LayerCase("decode-m1-n8-k64-r8", M=1, N=8, K=64, r=8, alpha=16.0, seed=114),
+    # 4104 = 128 x 32 + 8 rows: the last unit's 136 scale bytes end in an 8-byte tail
+    syn.LayerCase("decode-m9-n4104-k1088-r16", M=9, N=4104, K=1088, r=16, alpha=32.0, seed=115),
+    # 300 units: two or three per CTA (scale buffers reused, adapter product kept)
+    syn.LayerCase("decode-m3-n9600-k1024-r16", M=3, N=9600, K=1024, r=16, alpha=32.0, seed=116),
+    # longest rows on the small-M path (512 blocks of 64)
+    syn.LayerCase("decode-m2-n256-k32768-r8", M=2, N=256, K=32768, r=8, alpha=16.0, seed=117),
+    # rows longer than that: tensor-core path
+    syn.LayerCase("small-m4-n256-k33792-r8", M=4, N=256, K=33792, r=8, alpha=16.0, seed=118),
+    # adapter rank above the small-M kernel's limit: tensor-core path
     syn.LayerCase("decode-m1-n4096-k4096-r32", M=1, N=4096, K=4096, r=32, alpha=64.0, seed=110),
     # the 7B down projection at full size, 16 tokens, base only
     syn.LayerCase("decode-m16-n4096-k11008-r0", M=16, N=4096, K=11008, r=0, alpha=0.0, seed=111),
