@@ -12,34 +12,36 @@
 // Work split.  A unit is 32 W rows over all of K, so no partial sum ever leaves its
 // CTA.  One persistent CTA per SM takes a contiguous run of units.
 //
-// Data movement (two producer warps, eight consumer warps):
-//   - codes: a ring of 8 KB stages, each two TMA boxes of [32 rows x 128 B] (512 k)
-//     with the 128-byte swizzle, 8 stages deep: about 64 KB in flight per SM;
+// Data movement (two producer warps, eight consumer warps).  A stage is 1024 k:
+//   - codes: a ring of 16 KB stages, [4 chunks x 32 rows x 128 B] with the 128-byte
+//     swizzle, one 3-D TMA box per stage (four 2-D boxes when K is not a multiple of
+//     256), 3-6 stages deep.  TMA instructions are few and large because each costs
+//     a fixed few hundred nanoseconds of the SM's copy engine;
 //   - activations X (and, during a CTA's first unit, the adapter rows A): a second
-//     ring of [8 chunks x 8|16 rows x 128 B] swizzled boxes, 2-4 stages deep, fed by
-//     the second producer warp (these come from L2);
+//     ring of [16 chunks x M rows x 128 B] (and [16 x r x 128 B]) swizzled boxes, fed
+//     by the second producer warp (these come from L2);
 //   - block scales of a unit: one bulk copy of its 32 x K/64 bytes (contiguous in the
 //     packed layout) plus the unit's second-level steps, double-buffered per unit.
 //
-// Fragment mapping.  Consumer warp w takes block pair w % 4 of each stage (blocks
-// 2(w%4), 2(w%4)+1) and n8 groups 2(w/4), 2(w/4)+1 of the unit.  Lane (g, t) owns 32
-// consecutive weights: half t % 2 of block 2(w%4) + t/2, i.e. one 16-byte unit of
+// Fragment mapping.  Consumer warp w takes block pairs w % 4 and w % 4 + 4 of each
+// stage and n8 groups 2(w/4), 2(w/4)+1 of the unit.  For a block pair P, lane (g, t)
+// owns 32 consecutive weights: half t % 2 of block 2P + t/2, i.e. one 16-byte unit of
 // the swizzled code row, which it reads with one conflict-free 128-bit load.  MMA
 // column g is W row sigma(g) = 4 (g % 2) + g / 2 of the n8 group, chosen so that
 // the two rows read by each quarter-warp fall in different swizzle halves.  In
 // k-step j the lane supplies weights 4j .. 4j+3 of its 32 as B and the activations
 // at the same k positions as A; the MMA sums over its k slots in any order, so this
-// pairing only has to agree between A and B.
+// pairing only has to agree between A and B.  Each group keeps two accumulators (even
+// and odd k-steps) and the two groups alternate, so four independent MMA chains are
+// in flight per warp.
 //
 // The adapter product U = X A^T uses the same loop with the rows of A as extra n8
 // operands; every CTA computes it during its first unit and keeps it in shared
 // memory for the adapter term of all its units.
 //
 // Overlap with the preceding kernel (programmatic dependent launch): before waiting
-// on the preceding grid a CTA builds its table, initialises its barriers and
-// prefetches the code bytes of its first units into L2 (which is coherent);
-// every load into shared memory and every activation access follows
-// griddepcontrol.wait.
+// on the preceding grid a CTA only builds its table and initialises its barriers;
+// every load follows griddepcontrol.wait.
 #pragma once
 
 #include <cstdint>
@@ -52,16 +54,16 @@ namespace qlora {
 namespace dec {
 
 constexpr int kRows = 32;                       // W rows per unit
-constexpr int kStageK = 512;                    // k per pipeline stage
-constexpr int kStageBlocks = kStageK / 64;
+constexpr int kStageK = 1024;                   // k per pipeline stage
+constexpr int kStageBlocks = kStageK / 64;      // 16 blocks = 8 block pairs
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumers + 64;       // + two producer warps
 constexpr int kMaxRank = 16;                    // adapter ranks fused on this path
 constexpr int kMaxKB = 512;                     // 64-k blocks per row (n_in <= 32768)
-constexpr int kCodeStage = kRows * kStageK / 2; // 8 KB
+constexpr int kCodeStage = kRows * kStageK / 2; // 16 KB
 constexpr int kLutBytes = 256 * 32 * 4;         // one bf16x2 per byte value per lane
-constexpr int kMaxCodeStages = 8;
+constexpr int kMaxCodeStages = 6;
 constexpr int kMaxXaStages = 4;
 constexpr int kPartFloats = 4 * kRows * 16;     // [block pair][row][token]
 constexpr int kSmemLimit = 232448;
@@ -76,7 +78,7 @@ struct Params {
     int M, N, K, r;
     int units;               // ceil(N / 32)
     int dc, dx;              // ring depths (codes, activations)
-    int mbox, rbox;          // rows of the X and A boxes (8 or 16; rbox 0 without adapter)
+    int c3d;                 // codes map is 3-D (one box per stage)
     // byte offsets from the 1024-aligned shared-memory base
     int off_code, off_xa, xa_stage, off_sc, sc_stage, sc_q, off_part, off_upart, off_ufin, off_bars;
     float scaling;
@@ -90,9 +92,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -143,24 +142,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int u0 = static_cast<int>(int64_t(p.units) * blockIdx.x / gridDim.x);
     const int u1 = static_cast<int>(int64_t(p.units) * (blockIdx.x + 1) / gridDim.x);
     const int nu = u1 - u0;
-    const int nA = p.rbox / 8;                                        // adapter n8 groups
+    const int nA = p.r / 8;                                           // adapter n8 groups
 
     // 1. let the next kernel in the stream start launching
     pdl_launch_dependents();
 
-    // 2. byte -> bf16x2 (level[lo], level[hi]) table, one copy per lane
-    for (int e = threadIdx.x; e < 256; e += kThreads) {
-        float lo = 0.f, hi = 0.f;
+    // 2. byte -> bf16x2 (level[lo], level[hi]) table, one copy per lane.  Lane i holds
+    // level[i % 16] (constant-index reads keep the parameter block out of local
+    // memory); a thread writes 16-byte piece f % 8 of entry f / 8, so a warp's stores
+    // cover 512 contiguous bytes and no two lanes meet in a bank
+    {
+        float lvl = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {   // constant-index reads keep the parameter block out of local memory
-            if ((e & 15) == i) lo = p.level[i];
-            if ((e >> 4) == i) hi = p.level[i];
+        for (int i = 0; i < 16; ++i)
+            if ((lane & 15) == i) lvl = p.level[i];
+        const uint32_t base = smem_u32(smem);
+        for (int f0 = 0; f0 < 256 * 8; f0 += kThreads) {
+            const int f = f0 + static_cast<int>(threadIdx.x);
+            const int e = min(f, 256 * 8 - 1) >> 3;
+            const float lo = __shfl_sync(0xffffffffu, lvl, e & 15);
+            const float hi = __shfl_sync(0xffffffffu, lvl, e >> 4);
+            __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+            const uint32_t w = *reinterpret_cast<uint32_t *>(&v);
+            if (f < 256 * 8) sts128(base + f * 16, make_uint4(w, w, w, w));
         }
-        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-        const uint32_t w = *reinterpret_cast<uint32_t *>(&v);
-        const uint32_t base = smem_u32(smem) + e * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) sts128(base + c * 16, make_uint4(w, w, w, w));
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMaxCodeStages; ++i) { mbar_init(&code_full[i], 1); mbar_init(&code_empty[i], kConsumerWarps); }
@@ -169,17 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kConsumerWarps && lane == 0 && nu > 0) {
+    if (warp == kConsumerWarps && lane == 0) {
         tma_prefetch_desc(&tmC);
         tma_prefetch_desc(&tmX);
         if (nA > 0) tma_prefetch_desc(&tmA);
-        // the code rows of the first two units are contiguous: warm L2 with them
-        const int64_t row_bytes = p.K / 2;
-        const int64_t r0 = int64_t(u0) * kRows;
-        const int64_t r1 = min(int64_t(p.N), int64_t(min(u1, u0 + 2)) * kRows);
-        const uint8_t *src = p.codes + r0 * row_bytes;
-        for (int64_t off = 0, n = (r1 - r0) * row_bytes; off < n; off += 16384)
-            prefetch_l2_bulk(src + off, static_cast<uint32_t>((n - off < 16384 ? n - off : int64_t(16384))));
     }
     __syncthreads();
 
@@ -189,42 +187,52 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kConsumerWarps) {
         // ------------------------------------------------- code and scale producer
-        const int T = nu * nst;
-        int issued = 0, sc_issued = 0;
-        for (int i = 0; i < T; ++i) {
-            const int ui = i / nst, j = i - ui * nst;
+        int slot = 0, round = 0, issued = 0, sc_issued = 0;
+        bool ok = true;
+        for (int ui = 0; ui < nu && ok; ++ui) {
             const int u = u0 + ui;
-            if (j == 0) {   // this unit's block scales and second-level steps
-                const int sb = ui & 1;
-                if (ui >= 2 && !mbar_wait(&sc_empty[sb], ((ui >> 1) - 1) & 1, abort_flag)) break;
-                uint8_t *sq = smem + p.off_sc + sb * p.sc_stage;
-                float *s2 = reinterpret_cast<float *>(sq + p.sc_q);
-                const int rows = min(kRows, p.N - u * kRows);
-                const uint32_t bytes = static_cast<uint32_t>(rows * KB);
-                const uint32_t bulk = bytes & ~15u;
-                const int64_t fb0 = int64_t(u) * kRows * KB;   // first flat block of the unit
-                const int64_t g0 = fb0 >> 8, g1 = (fb0 + bytes - 1) >> 8;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sc_full[sb], bulk);
-                    if (bulk) bulk_g2s(sq, p.scales + fb0, bulk, &sc_full[sb]);
-                }
-                if (lane < 4) {
-                    const uint32_t off = bulk + 4u * lane;
-                    if (off < bytes) cp_async4(sq + off, p.scales + fb0 + off, min(4u, bytes - off));
-                }
-                for (int k = lane; k <= int(g1 - g0); k += 32) cp_async4(s2 + k, p.scales2 + g0 + k, 4u);
-                cp_async_arrive_noinc(&sc_full[sb]);
-                sc_issued = ui + 1;
-            }
-            const int slot = i % p.dc;
-            if (i >= p.dc && !mbar_wait(&code_empty[slot], ((i / p.dc) - 1) & 1, abort_flag)) break;
+            // this unit's block scales and second-level steps
+            const int sb = ui & 1;
+            if (ui >= 2 && !mbar_wait(&sc_empty[sb], ((ui >> 1) - 1) & 1, abort_flag)) break;
+            uint8_t *sq = smem + p.off_sc + sb * p.sc_stage;
+            float *s2 = reinterpret_cast<float *>(sq + p.sc_q);
+            const int rows = min(kRows, p.N - u * kRows);
+            const uint32_t bytes = static_cast<uint32_t>(rows * KB);
+            const uint32_t bulk = bytes & ~15u;
+            const int64_t fb0 = int64_t(u) * kRows * KB;   // first flat block of the unit
+            const int64_t g0 = fb0 >> 8, g1 = (fb0 + bytes - 1) >> 8;
             if (lane == 0) {
-                uint8_t *dst = smem + p.off_code + slot * kCodeStage;
-                mbar_arrive_expect_tx(&code_full[slot], kCodeStage);
-                tma_load_2d(dst, &tmC, &code_full[slot], j * (kStageK / 2), u * kRows);
-                tma_load_2d(dst + kCodeStage / 2, &tmC, &code_full[slot], j * (kStageK / 2) + 128, u * kRows);
+                mbar_arrive_expect_tx(&sc_full[sb], bulk);
+                if (bulk) bulk_g2s(sq, p.scales + fb0, bulk, &sc_full[sb]);
             }
-            issued = i + 1;
+            if (lane < 4) {
+                const uint32_t off = bulk + 4u * lane;
+                if (off < bytes) cp_async4(sq + off, p.scales + fb0 + off, min(4u, bytes - off));
+            }
+            for (int k = lane; k <= int(g1 - g0); k += 32) cp_async4(s2 + k, p.scales2 + g0 + k, 4u);
+            cp_async_arrive_noinc(&sc_full[sb]);
+            sc_issued = ui + 1;
+            // this unit's code stages
+            for (int j = 0; j < nst; ++j) {
+                if (round > 0 && !mbar_wait(&code_empty[slot], (round & 1) ^ 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    uint8_t *dst = smem + p.off_code + slot * kCodeStage;
+                    mbar_arrive_expect_tx(&code_full[slot], kCodeStage);
+                    if (p.c3d) {
+                        tma_load_3d(dst, &tmC, &code_full[slot], 0, u * kRows, j * (kStageK / 256));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < kStageK / 256; ++q)
+                            tma_load_2d(dst + q * (kRows * 128), &tmC, &code_full[slot], j * (kStageK / 2) + q * 128,
+                                        u * kRows);
+                    }
+                }
+                ++issued;
+                if (++slot == p.dc) { slot = 0; ++round; }
+            }
         }
         // nothing this warp issued may land after the CTA has exited
         if (lane == 0)
@@ -235,18 +243,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kConsumerWarps + 1) {
         // ------------------------------------------- activation (and adapter) producer
         if (lane == 0) {
-            const int T = nu * nst;
-            int issued = 0;
-            for (int i = 0; i < T; ++i) {
-                const int ui = i / nst, j = i - ui * nst;
-                const int slot = i % p.dx;
-                if (i >= p.dx && !mbar_wait(&xa_empty[slot], ((i / p.dx) - 1) & 1, abort_flag)) break;
-                const bool with_a = ui == 0 && nA > 0;
-                uint8_t *dst = smem + p.off_xa + slot * p.xa_stage;
-                mbar_arrive_expect_tx(&xa_full[slot], (p.mbox + (with_a ? p.rbox : 0)) * 1024);
-                tma_load_3d(dst, &tmX, &xa_full[slot], 0, 0, j * kStageBlocks);
-                if (with_a) tma_load_3d(dst + p.mbox * 1024, &tmA, &xa_full[slot], 0, 0, j * kStageBlocks);
-                issued = i + 1;
+            int slot = 0, round = 0, issued = 0;
+            bool ok = true;
+            for (int ui = 0; ui < nu && ok; ++ui) {
+                for (int j = 0; j < nst; ++j) {
+                    if (round > 0 && !mbar_wait(&xa_empty[slot], (round & 1) ^ 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const bool with_a = ui == 0 && nA > 0;
+                    uint8_t *dst = smem + p.off_xa + slot * p.xa_stage;
+                    mbar_arrive_expect_tx(&xa_full[slot], (p.M + (with_a ? p.r : 0)) * (kStageBlocks * 128));
+                    tma_load_3d(dst, &tmX, &xa_full[slot], 0, 0, j * kStageBlocks);
+                    if (with_a)
+                        tma_load_3d(dst + p.M * (kStageBlocks * 128), &tmA, &xa_full[slot], 0, 0, j * kStageBlocks);
+                    ++issued;
+                    if (++slot == p.dx) { slot = 0; ++round; }
+                }
             }
             for (int i = max(0, issued - p.dx); i < issued; ++i) mbar_drain(&xa_full[i % p.dx], (i / p.dx) & 1);
         }
@@ -261,20 +274,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lut = smem_u32(smem) + lane * 4;
     const uint32_t code_base = smem_u32(smem + p.off_code);
     const uint32_t xa_base = smem_u32(smem + p.off_xa);
-    float *part_all = reinterpret_cast<float *>(smem + p.off_part);
+    float *part = reinterpret_cast<float *>(smem + p.off_part);
     float *upart = reinterpret_cast<float *>(smem + p.off_upart);
     float *ufin = reinterpret_cast<float *>(smem + p.off_ufin);
     const bool tok0 = g < p.M, tok1 = NT > 1 && g + 8 < p.M;
-    const int chunk = 2 * pr + (t >> 1);               // 64-k chunk of the stage this lane reads
-    // byte offsets inside a stage: X row g (and g+8) of `chunk`, A row 8 gs + g, code row
-    const uint32_t x_off0 = uint32_t((chunk * p.mbox + g) * 128);
-    const uint32_t x_off1 = uint32_t((chunk * p.mbox + g + 8) * 128);
-    const uint32_t a_off = uint32_t(p.mbox * 1024 + (chunk * p.rbox + 8 * gs + g) * 128);
-    const uint32_t c_off = uint32_t((pr >> 1) * (kCodeStage / 2) + (((4 * (pr & 1) + t) ^ sg) << 4));
     const bool do_u = gs < nA;
     const int brow = ctid & 31;                         // epilogue row
+    const uint32_t u4 = 4 * (t & 1);                    // first 16-byte unit of this lane's half block
+    // per block pair h (pairs pr and pr + 4): the 64-k chunk this lane reads, its X lines
+    // (line = chunk * M + token; the swizzle XORs the unit with line % 8) and its code unit
+    int chunk[2];
+    uint32_t xl0[2], xl1[2], c_off[2], a_off[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        chunk[h] = 2 * (pr + 4 * h) + (t >> 1);
+        xl0[h] = uint32_t(chunk[h] * p.M + g);
+        xl1[h] = uint32_t(chunk[h] * p.M + g + 8);
+        c_off[h] = uint32_t(((pr >> 1) + 2 * h) * (kRows * 128) + (((4 * (pr & 1) + t) ^ sg) << 4));
+        a_off[h] = uint32_t(p.M * (kStageBlocks * 128) + (chunk[h] * p.r + 8 * gs + g) * 128);
+    }
 
-    int i = 0;   // stage counter
+    int cslot = 0, cph = 0, xslot = 0, xph = 0;
     for (int ui = 0; ui < nu; ++ui) {
         const int u = u0 + ui;
         const int n0 = u * kRows;
@@ -287,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bv0 = *reinterpret_cast<const uint4 *>(bp);
             if (p.r > 8) bv1 = *reinterpret_cast<const uint4 *>(bp + 8);
         }
-        mbar_wait(&sc_full[sb], (ui >> 1) & 1, abort_flag);
+        if (lane == 0) mbar_wait(&sc_full[sb], (ui >> 1) & 1, abort_flag);
+        __syncwarp();
         const uint32_t sq = smem_u32(smem + p.off_sc + sb * p.sc_stage);
         const uint32_t s2 = sq + p.sc_q;
         // flat block index of the unit's first block, modulo one second-level group: the
@@ -303,75 +324,87 @@ __global__ void __launch_bounds__(kThreads, 1)
             row_q[gg] = row * KB;
         }
 
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        float accU[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < nst; ++j, ++i) {
-            const int slot = i % p.dc, xslot = i % p.dx;
-            mbar_wait(&code_full[slot], (i / p.dc) & 1, abort_flag);
-            mbar_wait(&xa_full[xslot], (i / p.dx) & 1, abort_flag);
-            const int kb = j * kStageBlocks + chunk;
-            const bool kv = kb < KB;
-            const uint32_t xs = xa_base + uint32_t(xslot * p.xa_stage);
-            uint4 xw[4], xh[4];
+        float acc[2][2][4], accU[2][4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t sw = uint32_t(((4 * (t & 1) + q) ^ g) << 4);
-                xw[q] = tok0 ? lds128(xs + x_off0 + sw) : make_uint4(0, 0, 0, 0);
-                xh[q] = tok1 ? lds128(xs + x_off1 + sw) : make_uint4(0, 0, 0, 0);
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[0][a][b] = acc[1][a][b] = accU[a][b] = 0.f;
+        for (int j = 0; j < nst; ++j) {
+            if (lane == 0) {   // one lane polls; the warp barrier orders the others after it
+                mbar_wait(&code_full[cslot], cph, abort_flag);
+                mbar_wait(&xa_full[xslot], xph, abort_flag);
             }
-            const uint32_t cs = code_base + uint32_t(slot * kCodeStage) + c_off;
+            __syncwarp();
+            const uint32_t cs = code_base + uint32_t(cslot * kCodeStage);
+            const uint32_t xs = xa_base + uint32_t(xslot * p.xa_stage);
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                uint32_t sc = 0;
-                if (kv) {
-                    const uint32_t q = lds_u8(sq + uint32_t(row_q[gg] + kb));
-                    const float d = lds_f32(s2 + uint32_t(((fb_lo + row_q[gg] + kb) >> 8) << 2));
-                    __nv_bfloat162 s2b = __float2bfloat162_rn(__fmul_rn(static_cast<float>(q), d));
-                    sc = *reinterpret_cast<uint32_t *>(&s2b);
+            for (int h = 0; h < 2; ++h) {
+                const int kb = j * kStageBlocks + chunk[h];
+                const bool kv = kb < KB;
+                uint4 xw[4], xh[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    xw[q] = tok0 ? lds128(xs + xl0[h] * 128 + (((u4 + q) ^ (xl0[h] & 7)) << 4)) : make_uint4(0, 0, 0, 0);
+                    xh[q] = tok1 ? lds128(xs + xl1[h] * 128 + (((u4 + q) ^ (xl1[h] & 7)) << 4)) : make_uint4(0, 0, 0, 0);
                 }
-                const uint4 cw = lds128(cs + row_off[gg]);
-                const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint32_t sc[2];
+                uint4 cw[2];
+#pragma unroll
+                for (int gg = 0; gg < 2; ++gg) {
+                    sc[gg] = 0;
+                    if (kv) {
+                        const uint32_t q = lds_u8(sq + uint32_t(row_q[gg] + kb));
+                        const float d = lds_f32(s2 + uint32_t(((fb_lo + row_q[gg] + kb) >> 8) << 2));
+                        __nv_bfloat162 s2b = __float2bfloat162_rn(__fmul_rn(static_cast<float>(q), d));
+                        sc[gg] = *reinterpret_cast<uint32_t *>(&s2b);
+                    }
+                    cw[gg] = lds128(cs + c_off[h] + row_off[gg]);
+                }
 #pragma unroll
                 for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t word = cwv[jj >> 1];
-                    const uint32_t sh = 16 * (jj & 1);
-                    const uint32_t e0 = (word >> sh) & 0xFFu, e1 = (word >> (sh + 8)) & 0xFFu;
-                    const uint32_t b0 = bf16x2_mul(lds32(lut + (e0 << 7)), sc);
-                    const uint32_t b1 = bf16x2_mul(lds32(lut + (e1 << 7)), sc);
                     const uint4 &xa = xw[jj >> 1];
                     const uint4 &xb = xh[jj >> 1];
                     const uint32_t a0 = (jj & 1) ? xa.z : xa.x, a2 = (jj & 1) ? xa.w : xa.y;
                     const uint32_t a1 = (jj & 1) ? xb.z : xb.x, a3 = (jj & 1) ? xb.w : xb.y;
-                    mma_bf16_16816(acc[gg], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, b0, b1);
+#pragma unroll
+                    for (int gg = 0; gg < 2; ++gg) {
+                        const uint32_t cwv[4] = {cw[gg].x, cw[gg].y, cw[gg].z, cw[gg].w};
+                        const uint32_t word = cwv[jj >> 1];
+                        const uint32_t sh = 16 * (jj & 1);
+                        const uint32_t e0 = (word >> sh) & 0xFFu, e1 = (word >> (sh + 8)) & 0xFFu;
+                        const uint32_t b0 = bf16x2_mul(lds32(lut + (e0 << 7)), sc[gg]);
+                        const uint32_t b1 = bf16x2_mul(lds32(lut + (e1 << 7)), sc[gg]);
+                        mma_bf16_16816(acc[gg][jj & 1], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, b0, b1);
+                    }
                 }
-            }
-            if (first && do_u) {
+                if (first && do_u) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t sw = uint32_t(((4 * (t & 1) + q) ^ g) << 4);
-                    const uint4 aw = lds128(xs + a_off + sw);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 aw = lds128(xs + a_off[h] + (((u4 + q) ^ g) << 4));
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint4 &xa = xw[q];
-                        const uint4 &xb = xh[q];
-                        const uint32_t a0 = h ? xa.z : xa.x, a2 = h ? xa.w : xa.y;
-                        const uint32_t a1 = h ? xb.z : xb.x, a3 = h ? xb.w : xb.y;
-                        mma_bf16_16816(accU, a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, h ? aw.z : aw.x,
-                                       h ? aw.w : aw.y);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const uint4 &xa = xw[q];
+                            const uint4 &xb = xh[q];
+                            const uint32_t a0 = hh ? xa.z : xa.x, a2 = hh ? xa.w : xa.y;
+                            const uint32_t a1 = hh ? xb.z : xb.x, a3 = hh ? xb.w : xb.y;
+                            mma_bf16_16816(accU[hh], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, hh ? aw.z : aw.x,
+                                           hh ? aw.w : aw.y);
+                        }
                     }
                 }
             }
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&code_empty[slot]);
+                mbar_arrive(&code_empty[cslot]);
                 mbar_arrive(&xa_empty[xslot]);
             }
+            if (++cslot == p.dc) { cslot = 0; cph ^= 1; }
+            if (++xslot == p.dx) { xslot = 0; xph ^= 1; }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sc_empty[sb]);
 
-        // partial sums of this block pair -> part[pr][row][token]
-        float *part = part_all + sb * kPartFloats;
+        // partial sums of block pairs pr, pr + 4 -> part[pr][row][token]
         float *pb = part + pr * kRows * 16;
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
@@ -379,18 +412,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c0 = 2 * t, c1 = 2 * t + 1;
             const int R0 = 8 * grp + (((c0 & 1) << 2) | (c0 >> 1));
             const int R1 = 8 * grp + (((c1 & 1) << 2) | (c1 >> 1));
-            pb[R0 * 16 + g] = acc[gg][0];
-            pb[R1 * 16 + g] = acc[gg][1];
-            pb[R0 * 16 + g + 8] = acc[gg][2];
-            pb[R1 * 16 + g + 8] = acc[gg][3];
+            pb[R0 * 16 + g] = acc[gg][0][0] + acc[gg][1][0];
+            pb[R1 * 16 + g] = acc[gg][0][1] + acc[gg][1][1];
+            pb[R0 * 16 + g + 8] = acc[gg][0][2] + acc[gg][1][2];
+            pb[R1 * 16 + g + 8] = acc[gg][0][3] + acc[gg][1][3];
         }
         if (first && do_u) {
             float *ub = upart + pr * 256;
             const int j0 = 8 * gs + 2 * t;
-            ub[g * 16 + j0] = accU[0];
-            ub[g * 16 + j0 + 1] = accU[1];
-            ub[(g + 8) * 16 + j0] = accU[2];
-            ub[(g + 8) * 16 + j0 + 1] = accU[3];
+            ub[g * 16 + j0] = accU[0][0] + accU[1][0];
+            ub[g * 16 + j0 + 1] = accU[0][1] + accU[1][1];
+            ub[(g + 8) * 16 + j0] = accU[0][2] + accU[1][2];
+            ub[(g + 8) * 16 + j0 + 1] = accU[0][3] + accU[1][3];
         }
         consumer_sync();
         if (first && p.r > 0) {
@@ -400,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.U_save && blockIdx.x == 0) {
                 for (int e = ctid; e < p.M * p.r; e += kConsumers) {
                     const int m = e / p.r, jr = e - m * p.r;
-                    __nv_bfloat16 h = __float2bfloat16_rn(ufin[m * 16 + jr]);
-                    p.U_save[e] = *reinterpret_cast<uint16_t *>(&h);
+                    __nv_bfloat16 hv = __float2bfloat16_rn(ufin[m * 16 + jr]);
+                    p.U_save[e] = *reinterpret_cast<uint16_t *>(&hv);
                 }
             }
         }
@@ -422,10 +455,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                __nv_bfloat16 h = __float2bfloat16_rn(fmaf(p.scaling, l, base));
-                p.Y[int64_t(m) * p.N + n] = *reinterpret_cast<uint16_t *>(&h);
+                __nv_bfloat16 hv = __float2bfloat16_rn(fmaf(p.scaling, l, base));
+                p.Y[int64_t(m) * p.N + n] = *reinterpret_cast<uint16_t *>(&hv);
             }
         }
+        if (ui + 1 < nu) consumer_sync();   // the next unit rewrites the partial sums
     }
 }
 

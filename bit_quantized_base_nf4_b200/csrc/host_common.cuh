@@ -167,6 +167,26 @@ static qlora_status make_tmap_chunks(CUtensorMap *map, const void *base, uint64_
     return QLORA_OK;
 }
 
+// 3-D map viewing packed codes, u8 [rows, K/2], as [K/256 chunks][rows][128 B]: one box
+// = `depth` consecutive 128-byte chunks of `box_rows` rows, each a 128-byte-swizzled
+// [box_rows x 128 B] tile, stored chunk after chunk.  K must be a multiple of 256.
+static qlora_status make_tmap_code_chunks(CUtensorMap *map, const void *codes, uint64_t rows, uint64_t K,
+                                          uint32_t box_rows, uint32_t depth) {
+    auto fn = encode_fn();
+    if (!fn) return fail(QLORA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    cuuint64_t dims[3] = {128, rows, K / 256};
+    cuuint64_t strides[2] = {K / 2, 128};
+    cuuint32_t box[3] = {128, box_rows, depth};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(codes), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(QLORA_ERR_CUDA, "cuTensorMapEncodeTiled (codes, 3-D) failed (%d) rows=%llu K=%llu", int(r),
+                    (unsigned long long)rows, (unsigned long long)K);
+    return QLORA_OK;
+}
+
 // ------------------------------------------------------------------ device checks
 static qlora_status require_sm100() {
     int dev = 0;

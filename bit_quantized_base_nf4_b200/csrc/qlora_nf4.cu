@@ -126,27 +126,24 @@ int pair_token_tile(int64_t M) {
     const int64_t bn = ceil_div(ceil_div(M, tiles), 32) * 32;
     return static_cast<int>(std::max<int64_t>(32, std::min<int64_t>(256, bn)));
 }
-// Small-M forward: the weight-streaming warp-MMA kernel (decode_mma.cuh), which
-// needs no workspace, for up to 16 tokens, adapter ranks up to 16 and n_in up to 32768.
-bool use_decode(int64_t M, int64_t K, int r) { return M <= 16 && r <= dec::kMaxRank && K / 64 <= dec::kMaxKB; }
-
-// Shared-memory plan of the small-M kernel: table, code ring, activation ring, two
-// scale buffers, partial sums, barriers.  The rings are as deep as the 227 KB allow.
+// Shared-memory plan of the small-M kernel (decode_mma.cuh): table, code ring,
+// activation ring, two scale buffers, partial sums, barriers.  The rings are as deep
+// as the 227 KB allow; a shape whose shallowest rings do not fit is not planned.
 struct DecodePlan {
     dec::Params p;
     int smem;
+    bool fits;
 };
 DecodePlan plan_decode(int64_t M, int64_t K, int r) {
     DecodePlan d{};
     dec::Params &p = d.p;
     const int KB = static_cast<int>(K / 64);
-    p.mbox = M <= 8 ? 8 : 16;
-    p.rbox = r == 0 ? 0 : (r <= 8 ? 8 : 16);
     const int sc_q = (dec::kRows * KB + 16 + 15) & ~15;
     const int s2_floats = ((dec::kRows * KB) / 256 + 2 + 3) & ~3;
     p.sc_q = sc_q;
     p.sc_stage = (sc_q + 4 * s2_floats + 127) & ~127;
-    p.xa_stage = (p.mbox + p.rbox) * 1024;
+    p.xa_stage = static_cast<int>((M + r) * dec::kStageBlocks * 128);
+    p.c3d = (K % 256 == 0) ? 1 : 0;
     auto total = [&](int dc, int dx) {
         p.dc = dc;
         p.dx = dx;
@@ -154,19 +151,25 @@ DecodePlan plan_decode(int64_t M, int64_t K, int r) {
         p.off_xa = p.off_code + dc * dec::kCodeStage;
         p.off_sc = p.off_xa + dx * p.xa_stage;
         p.off_part = p.off_sc + 2 * p.sc_stage;
-        p.off_upart = p.off_part + 2 * dec::kPartFloats * 4;
+        p.off_upart = p.off_part + dec::kPartFloats * 4;
         p.off_ufin = p.off_upart + 4 * 256 * 4;
         p.off_bars = p.off_ufin + 256 * 4;
         const int bars = (2 * dec::kMaxCodeStages + 2 * dec::kMaxXaStages + 4) * 8 + 16;
         return 1024 + p.off_bars + bars;   // + alignment slack of the dynamic base
     };
     int dc = dec::kMaxCodeStages, dx = dec::kMaxXaStages;
-    while (total(dc, dx) > dec::kSmemLimit && (dx > 2 || dc > 4)) {
+    while (total(dc, dx) > dec::kSmemLimit && (dx > 2 || dc > 3)) {
         if (dx > 2) --dx;
         else --dc;
     }
     d.smem = total(dc, dx);
+    d.fits = d.smem <= dec::kSmemLimit;
     return d;
+}
+// Small-M forward: the weight-streaming warp-MMA kernel, which needs no workspace,
+// for up to 16 tokens, adapter ranks up to 16 and n_in up to 32768 (when its rings fit).
+bool use_decode(int64_t M, int64_t K, int r) {
+    return M <= 16 && r <= dec::kMaxRank && K / 64 <= dec::kMaxKB && plan_decode(M, K, r).fits;
 }
 size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (use_decode(M, K, r)) return 0;
@@ -372,8 +375,6 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
 
     if (use_decode(M, K, r)) {
         DecodePlan d = plan_decode(M, K, r);
-        if (d.smem > dec::kSmemLimit)
-            return fail(QLORA_ERR_SHAPE, "n_in (%lld) too large for the small-M path", (long long)K);
         dec::Params &p = d.p;
         p.codes = w->codes;
         p.scales = w->scales;
@@ -389,12 +390,14 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         p.scaling = scaling;
         const Codebook &cbd = codebook();
         for (int i = 0; i < 16; ++i) p.level[i] = cbd.level[i];
-        // codes as u8 [N, K/2]: [32 rows x 128 B] boxes; X and A as [K/64][rows][64] bf16 chunks
+        // codes as u8 [N, K/2] in [32 rows x 128 B] boxes (3-D: four 256-k chunks per box);
+        // X and A as [K/64][rows][64] bf16 chunks, sixteen chunks per box
         CUtensorMap tmC, tmX, tmA;
-        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, dec::kRows, 128,
-                            CU_TENSOR_MAP_SWIZZLE_128B));
-        QL_TRY(make_tmap_chunks(&tmX, X, M, K, p.mbox, dec::kStageBlocks));
-        if (r > 0) QL_TRY(make_tmap_chunks(&tmA, A, r, K, p.rbox, dec::kStageBlocks));
+        if (p.c3d) QL_TRY(make_tmap_code_chunks(&tmC, w->codes, N, K, dec::kRows, dec::kStageK / 256));
+        else QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, dec::kRows, 128,
+                                 CU_TENSOR_MAP_SWIZZLE_128B));
+        QL_TRY(make_tmap_chunks(&tmX, X, M, K, static_cast<uint32_t>(M), dec::kStageBlocks));
+        if (r > 0) QL_TRY(make_tmap_chunks(&tmA, A, r, K, static_cast<uint32_t>(r), dec::kStageBlocks));
         else tmA = tmX;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(p.units, sm_count())));
