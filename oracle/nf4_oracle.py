@@ -32,6 +32,8 @@ Readings adopted where the pages are silent:
 * Dequant: s_b = RN32(q_b * d_g), w' = RN32(c[code] * s_b).
 * Layer: Y = X W'^T + s (X A^T) B^T, dX = dY W' + s (dY B) A,
   dA = s (dY B)^T X, dB = s dY^T (X A^T), no gradient for W0.
+* Merge: m = bf16(RN32(bf16(w') + s sum_j B[n, j] A[j, k])), sum and product in
+  float64 with j ascending, then the NF4 + double-quant encode of m.
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
 tests/test_oracle_pins.py against a fact other than itself (a printed worked
@@ -314,6 +316,39 @@ def lora_linear_fwd_rows(w_deq, x, a, b, scaling: float, rows):
 # ---------------------------------------------------------------------------
 # Tolerance used for every floating-point output (the layer's stated bar)
 # ---------------------------------------------------------------------------
+
+# ---------------------------------------------------------------------------
+# Merging the adapter back into the quantized base ("Course notes" page, §3.3:
+# dequantize W to BF16, merge at high precision, quantize again; "Training LoRA
+# directly on GGUF quantized weights" page, §3.3 and §4.3: merge the dequantized
+# base and the LoRA into bf16, then rerun the quantization, with one rounding in
+# the merge and one in the requantization; merge formula W' = W + B A from the
+# "Course notes" page, §3.2)
+# ---------------------------------------------------------------------------
+
+def lora_merge_bf16(codes, q, d, n_out: int, n_in: int, a, b, scaling: float) -> np.ndarray:
+    """The merged base as float32 holding bf16 values:
+    m = bf16(RN32(bf16(w') + s * sum_j B[n, j] A[j, k])).
+
+    The dequantized base is taken to bf16 first (the pages' "dequantize to BF16").
+    The adapter product and the add are done in float64 ("high precision"), j in
+    ascending order; bf16 x bf16 products are exact in float64.  The float64 sum is
+    rounded to float32 and then to bf16, the precision the merged base is kept in.
+    a [r, K] and b [N, r] are the bf16 adapter factors (any r >= 0)."""
+    w = dequant(codes, q, d, n_out * n_in).reshape(n_out, n_in)
+    wb = bf16_round(w).astype(np.float64)
+    acc = np.zeros((n_out, n_in), np.float64)
+    a64, b64 = _f64(a), _f64(b)
+    for j in range(a64.shape[0] if a64.size else 0):
+        acc = acc + np.outer(b64[:, j], a64[j, :])
+    m = wb + np.float64(np.float32(scaling)) * acc
+    return bf16_round(m.astype(np.float32))
+
+
+def lora_merge_requant(codes, q, d, n_out: int, n_in: int, a, b, scaling: float) -> dict:
+    """W'' = quant(merged base): the NF4 + double-quant encode of lora_merge_bf16."""
+    return quantize_nf4_dq(lora_merge_bf16(codes, q, d, n_out, n_in, a, b, scaling))
+
 
 def rel_errors(got, ref):
     """(normwise ||got-ref||_F/||ref||_F, max over rows of max|err| / max(max|ref_row|, 1e-6))."""

@@ -10,6 +10,7 @@ import json
 import math
 import os
 import statistics
+import struct
 
 import numpy as np
 import pytest
@@ -434,3 +435,118 @@ def test_dq_ratio_and_products_are_correctly_rounded():
     w = O.dequant(O.pack_codes(codes), q, d)
     for i in range(0, w.size, 37):
         assert w[i] == _rn32_exact(Fraction(float(book[codes[i]])) * Fraction(float(s[i // 64])))
+
+
+# ------------------------------------------------ LoRA merge and requantize
+
+def _f32_rn(x):
+    """IEEE float32 round-to-nearest of a Python float, through struct packing."""
+    return struct.unpack("<f", struct.pack("<f", x))[0]
+
+
+def _bf16_rn(x):
+    """bfloat16 round-to-nearest-even of a float32 value, on its bit pattern as an int."""
+    u = struct.unpack("<I", struct.pack("<f", x))[0]
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return struct.unpack("<f", struct.pack("<I", u & 0xFFFFFFFF))[0]
+
+
+def _merge_case(n_out, n_in, r, seed, w_std=0.02):
+    rng = np.random.default_rng(seed)
+    W = rng.normal(0, w_std, (n_out, n_in)).astype(np.float32)
+    ref = O.quantize_nf4_dq(W)
+    A = O.bf16_round(rng.normal(0, 1.0 / n_in, (r, n_in)).astype(np.float32))
+    B = O.bf16_round(rng.normal(0, 0.01, (n_out, r)).astype(np.float32))
+    return ref, A, B
+
+
+def test_merge_brute_force_python():
+    # pins lora_merge_bf16 by pure-Python loops: per element, the bf16 base, the
+    # float64 sum over j in ascending order, then float32 and bf16 rounding by struct
+    n_out, n_in, r, s = 8, 64, 8, 2.0
+    ref, A, B = _merge_case(n_out, n_in, r, seed=71)
+    got = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s)
+    book = [float(v) for v in O.nf4_codebook()]
+    for n in range(n_out):
+        for k in range(n_in):
+            e = n * n_in + k
+            byte = int(ref["codes"][e // 2])
+            code = (byte & 15) if e % 2 == 0 else (byte >> 4)
+            blk = e // 64
+            sb = _f32_rn(float(ref["scales"][blk]) * float(ref["scales2"][blk // 256]))
+            w = _f32_rn(book[code] * sb)
+            acc = 0.0
+            for j in range(r):
+                acc = acc + float(B[n, j]) * float(A[j, k])
+            want = _bf16_rn(_f32_rn(_bf16_rn(w) + float(np.float32(s)) * acc))
+            assert float(got[n, k]) == want, (n, k)
+
+
+def test_merge_rank_one_single_row_closed_form():
+    # B = unit column at row n0: only row n0 moves, by bf16(RN32(bf16(w') + s a_k))
+    n_out, n_in, s, n0 = 16, 128, 0.75, 5
+    ref, _, _ = _merge_case(n_out, n_in, 1, seed=72)
+    rng = np.random.default_rng(73)
+    a = O.bf16_round(rng.normal(0, 0.05, (1, n_in)).astype(np.float32))
+    b = np.zeros((n_out, 1), np.float32)
+    b[n0, 0] = 1.0
+    got = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, a, b, s)
+    base = O.bf16_round(O.dequant(ref["codes"], ref["scales"], ref["scales2"])).reshape(n_out, n_in)
+    others = np.arange(n_out) != n0
+    assert np.array_equal(got[others], base[others])
+    for k in range(n_in):
+        assert float(got[n0, k]) == _bf16_rn(_f32_rn(float(base[n0, k]) + s * float(a[0, k])))
+
+
+def test_merge_of_zero_base_is_the_exact_adapter_product():
+    # W0 = 0 encodes to code 7 and zero scales, so the base dequantizes to 0; with
+    # power-of-two factors s B A is exact in bf16, the merge returns it unchanged and
+    # the requantization equals the plain encode of s B A
+    n_out, n_in, r, s = 32, 256, 8, 0.5
+    ref = O.quantize_nf4_dq(np.zeros((n_out, n_in), np.float32))
+    rng = np.random.default_rng(74)
+    A = (2.0 ** rng.integers(-6, 0, (r, n_in))).astype(np.float32) * rng.choice([-1, 1], (r, n_in))
+    B = np.zeros((n_out, r), np.float32)
+    B[np.arange(n_out), rng.integers(0, r, n_out)] = (2.0 ** rng.integers(-4, 0, n_out)).astype(np.float32)
+    prod = s * B.astype(np.float64) @ A.astype(np.float64)
+    got = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s)
+    assert np.array_equal(got.astype(np.float64), prod)
+    out = O.lora_merge_requant(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s)
+    direct = O.quantize_nf4_dq(prod.astype(np.float32))
+    for key in ("codes", "scales", "scales2"):
+        assert np.array_equal(out[key], direct[key])
+
+
+def test_merge_close_to_float64_definition():
+    # the merged base is W' + s B A up to the bf16 roundings (two, each 2^-9 relative)
+    n_out, n_in, r, s = 64, 512, 16, 2.0
+    ref, A, B = _merge_case(n_out, n_in, r, seed=75)
+    got = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s).astype(np.float64)
+    w = O.dequant(ref["codes"], ref["scales"], ref["scales2"]).reshape(n_out, n_in).astype(np.float64)
+    exact = w + s * B.astype(np.float64) @ A.astype(np.float64)
+    assert np.all(np.abs(got - exact) <= np.abs(w) * 2.0 ** -8 + np.abs(exact) * 2.0 ** -8 + 1e-30)
+    # the adapter term is really in it: with factors large enough that s B A is far
+    # above the bf16 rounding of the base, the merged change is s B A
+    # (at the realistic adapter scale the two are comparable, the merge loss the
+    # GGUF page warns about)
+    rng = np.random.default_rng(77)
+    A2 = O.bf16_round(rng.normal(0, 1.0 / 16, (r, n_in)).astype(np.float32))
+    B2 = O.bf16_round(rng.normal(0, 0.1, (n_out, r)).astype(np.float32))
+    got2 = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A2, B2, s).astype(np.float64)
+    delta = got2 - O.bf16_round(w.astype(np.float32)).astype(np.float64)
+    lora = s * B2.astype(np.float64) @ A2.astype(np.float64)
+    assert np.linalg.norm(delta - lora) < 0.05 * np.linalg.norm(lora)
+
+
+def test_merge_requant_round_trip_bound():
+    # the requantized merge obeys the encode's per-block bound around the merged base
+    n_out, n_in, r, s = 64, 512, 8, 2.0
+    ref, A, B = _merge_case(n_out, n_in, r, seed=76)
+    m = O.lora_merge_bf16(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s).reshape(-1)
+    out = O.lora_merge_requant(ref["codes"], ref["scales"], ref["scales2"], n_out, n_in, A, B, s)
+    back = O.dequant(out["codes"], out["scales"], out["scales2"]).astype(np.float64)
+    a = out["absmax"].astype(np.float64)
+    sb = O.dequant_scales(out["scales"], out["scales2"]).astype(np.float64)
+    half_gap = float(np.max(np.diff(O.nf4_codebook().astype(np.float64)))) / 2
+    bound = np.repeat(a * half_gap + np.abs(a - sb), 64) * (1 + 1e-6) + 1e-30
+    assert np.all(np.abs(back - m.astype(np.float64)) <= bound)
