@@ -326,6 +326,48 @@ def quantize_pass(dev, steps, warmup):
             "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
 
 
+# ----------------------------------------------------------------------------- merge pass
+
+def merge_pass(dev, steps, warmup):
+    """LoRA merge + requantize (dequant to bf16, add s B A in float64, round to bf16,
+    NF4 + DQ encode) of the 7B attention projection (4096 x 4096, r = 8) and the 70B FFN
+    up projection (28672 x 8192, r = 64).  GB/s on the algorithmic bytes: packed weight
+    in and out plus A and B; "moved" adds the float32 merged base the encode reads
+    back (written once, read once)."""
+    import torch
+    import bit_quantized_base_nf4_b200 as q
+    from bit_quantized_base_nf4_b200 import synthetic as syn
+    out = {}
+    for name, N, K, r, std in (("7B attn 4096x4096 r=8", 4096, 4096, 8, 0.02),
+                               ("70B FFN up 28672x8192 r=64", 28672, 8192, 64, 0.015)):
+        g = torch.Generator(device=dev)
+        g.manual_seed(5200 + r)
+        W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32) * std
+        w = q.NF4Weight.empty(N, K, device=dev)
+        q.qlora_quantize_nf4_dq(W, w)
+        scratch = W   # the merged base overwrites the fp32 input, no longer needed
+        A = syn.normal_bf16((r, K), 1.0 / K, 5300 + r).to(dev)
+        B = syn.normal_bf16((N, r), 0.01, 5400 + r).to(dev)
+        w_out = q.NF4Weight.empty(N, K, device=dev)
+        for _ in range(warmup):
+            q.qlora_lora_merge_requant(w, A, B, r, 16.0 / r, scratch, w_out)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            q.qlora_lora_merge_requant(w, A, B, r, 16.0 / r, scratch, w_out)
+        b.record()
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status()
+        ms = a.elapsed_time(b) / steps
+        algo = 2 * q.qlora_packed_bytes(N * K) + 2 * r * (N + K)
+        moved = algo + 8 * N * K
+        out[name] = {"ms": ms, "GB/s": algo / (ms * 1e-3) / 1e9, "moved_GB/s": moved / (ms * 1e-3) / 1e9,
+                     "moved_frac_of_hbm": moved / (ms * 1e-3) / 1e9 / peaks()["hbm_gbs"]}
+        del W, scratch, w, w_out, A, B
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------------------- CUDA leg
 
 def run_ours(args, case):
@@ -478,6 +520,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode-sweep GB/s measurement")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode sweep (prints its JSON)")
     ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS)
+    ap.add_argument("--merge-only", action="store_true", help="run only the merge + requantize pass (prints its JSON)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -485,6 +528,11 @@ def main():
     case = syn.attn7b_case()
     if args.impl == "reference":
         run_reference(args, case)
+    elif args.merge_only:
+        import torch
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"merge": merge_pass(dev, args.steps, args.warmup)}), flush=True)
     elif args.decode_only:
         import torch
         dev = torch.device("cuda", 0)

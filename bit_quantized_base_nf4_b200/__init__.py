@@ -16,6 +16,7 @@ import torch
 from . import _capi
 
 __all__ = ["NF4Weight", "qlora_packed_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq", "qlora_dequant",
+           "qlora_lora_merge_requant",
            "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
            "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
            "qlora_sync_status", "QloraError"]
@@ -91,6 +92,23 @@ def qlora_dequant(weight: NF4Weight, out: torch.Tensor, stream=None) -> None:
     s = weight.c_struct()
     _capi.check("qlora_dequant", _lib().qlora_dequant(ctypes.byref(s), _ptr(out), int(out.dtype == torch.bfloat16),
                                                       _stream(stream)))
+
+
+def qlora_lora_merge_requant(weight: NF4Weight, A, B, r: int, scaling: float, W_scratch: torch.Tensor,
+                             out: NF4Weight, stream=None) -> None:
+    """Merge the adapter into the base and quantize again into `out` (may be `weight`);
+    W_scratch is a float32 [n_out, n_in] device tensor that receives the merged base."""
+    _need(W_scratch, torch.float32, (weight.n_out, weight.n_in), "W_scratch")
+    if (out.n_out, out.n_in) != (weight.n_out, weight.n_in):
+        raise ValueError("out must have the shape of weight")
+    if r:
+        _need(A, torch.bfloat16, (r, weight.n_in), "A")
+        _need(B, torch.bfloat16, (weight.n_out, r), "B")
+    s_in, s_out = weight.c_struct(), out.c_struct()
+    _capi.check("qlora_lora_merge_requant",
+                _lib().qlora_lora_merge_requant(ctypes.byref(s_in), _ptr(A) if r else None, _ptr(B) if r else None,
+                                                int(r), float(scaling), _ptr(W_scratch), ctypes.byref(s_out),
+                                                _stream(stream)))
 
 
 def qlora_workspace_bytes(M: int, N: int, K: int, r: int) -> int:

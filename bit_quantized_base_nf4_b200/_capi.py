@@ -29,6 +29,7 @@ SIGNATURES = {
     "qlora_nf4_codebook": (_int, [ctypes.POINTER(ctypes.c_float)]),
     "qlora_quantize_nf4_dq": (_int, [_vp, _WP, _vp]),
     "qlora_dequant": (_int, [_WP, _vp, _int, _vp]),
+    "qlora_lora_merge_requant": (_int, [_WP, _vp, _vp, _int, _f32, _vp, _WP, _vp]),
     "qlora_workspace_bytes": (_sz, [_i64, _i64, _i64, _int]),
     "qlora_lora_linear_fwd": (_int, [_WP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_lora_linear_fwd_static_ws": (_int, [_WP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp]),

@@ -358,6 +358,28 @@ qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16
     return launch_check("nf4_dequant_kernel launch");
 }
 
+qlora_status qlora_lora_merge_requant(const qlora_nf4_weight *w_in, const qlora_bf16 *A, const qlora_bf16 *B, int r,
+                                      float scaling, float *W_scratch, const qlora_nf4_weight *w_out, void *stream) {
+    QL_TRY(check_weight(w_in));
+    QL_TRY(check_weight(w_out));
+    if (w_out->n_out != w_in->n_out || w_out->n_in != w_in->n_in)
+        return fail(QLORA_ERR_SHAPE, "w_out must have the shape of w_in");
+    QL_TRY(check_rank(r, scaling, A, B));
+    if (!W_scratch) return fail(QLORA_ERR_ARG, "W_scratch is NULL");
+    if (!aligned16(W_scratch)) return fail(QLORA_ERR_ALIGN, "W_scratch must be 16-byte aligned");
+    QL_TRY(require_sm100());
+    // x: the code words of a row (8 weights each); y: rows, about 16 CTAs per SM in all
+    const int64_t gx = std::min<int64_t>(ceil_div(w_in->n_in / 8, 256), 32);
+    const int64_t gy = std::min<int64_t>(w_in->n_out, std::max<int64_t>(1, int64_t(sm_count()) * 16 / gx));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    nf4_lora_merge_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
+        w_in->codes, w_in->scales, w_in->scales2, r > 0 ? reinterpret_cast<const uint16_t *>(A) : nullptr,
+        r > 0 ? reinterpret_cast<const uint16_t *>(B) : nullptr, r, r > 0 ? scaling : 0.f, w_in->n_out, w_in->n_in,
+        W_scratch, codebook_arg());
+    QL_TRY(launch_check("nf4_lora_merge_kernel launch"));
+    return qlora_quantize_nf4_dq(W_scratch, w_out, stream);
+}
+
 qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *X, int64_t M, const qlora_bf16 *A,
                                    const qlora_bf16 *B, int r, float scaling, qlora_bf16 *Y, qlora_bf16 *U_save,
                                    void *ws, size_t ws_bytes, void *stream) {

@@ -105,6 +105,21 @@ qlora_status qlora_quantize_nf4_dq(const float *W, const qlora_nf4_weight *w, vo
  * (out_is_bf16 = 1).  Bit-exact. */
 qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16, void *stream);
 
+/* Merge the adapter into the base and quantize again (the deployment step of
+ * the "Course notes: LLM basics and quantized fine-tuning" page, section 3.3,
+ * and of the GGUF page, sections 3.3 and 4.3: dequantize the base to bf16,
+ * merge at high precision, rerun the quantization):
+ *   m[n, k] = bf16(fp32(bf16(w'[n, k]) + scaling * sum_j B[n, j] A[j, k])),
+ * the sum and the add in float64 with j ascending, then w_out = the NF4 +
+ * double-quant encode of m (as qlora_quantize_nf4_dq).  A [r, K] and B [N, r]
+ * are bf16 with the rank rules of qlora_lora_linear_fwd; r = 0 requantizes
+ * bf16(w').  W_scratch: caller-owned device float32 [n_out, n_in] (4 * numel
+ * bytes); it holds m when the call completes.  w_out has the shape of w_in and
+ * may be w_in itself (the merge reads all of w_in before the encode writes).
+ * Bit-exact. */
+qlora_status qlora_lora_merge_requant(const qlora_nf4_weight *w_in, const qlora_bf16 *A, const qlora_bf16 *B, int r,
+                                      float scaling, float *W_scratch, const qlora_nf4_weight *w_out, void *stream);
+
 /* Scratch bytes needed by qlora_lora_linear_fwd / qlora_lora_linear_bwd_dx for
  * these sizes (N = n_out, K = n_in).  0 is never returned for valid sizes. */
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);

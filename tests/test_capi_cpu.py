@@ -95,6 +95,16 @@ def test_validation_rejects_before_launch(lib):
     # misaligned activations
     assert lib.qlora_lora_linear_fwd(ctypes.byref(w), ctypes.c_void_p(0x10002), 16, A, B, 8, 2.0, Y, None, ws,
                                      1 << 20, None) == 3
+    # merge + requantize argument rules
+    sc = ctypes.c_void_p(0x80000)
+    w2 = _w(n_out=128)
+    assert lib.qlora_lora_merge_requant(ctypes.byref(w), A, B, 8, 2.0, sc, ctypes.byref(w2), None) == 2
+    assert "shape" in _err(lib)
+    assert lib.qlora_lora_merge_requant(ctypes.byref(w), A, B, 12, 2.0, sc, ctypes.byref(w), None) == 2
+    assert lib.qlora_lora_merge_requant(ctypes.byref(w), None, B, 8, 2.0, sc, ctypes.byref(w), None) == 1
+    assert lib.qlora_lora_merge_requant(ctypes.byref(w), A, B, 8, 2.0, None, ctypes.byref(w), None) == 1
+    assert lib.qlora_lora_merge_requant(ctypes.byref(w), A, B, 8, 2.0, ctypes.c_void_p(0x80004), ctypes.byref(w),
+                                        None) == 3
     # grad_AB argument rules
     dA, dB = ctypes.c_void_p(0x60000), ctypes.c_void_p(0x70000)
     assert lib.qlora_lora_grad_AB(X, Y, A, B, 16, 256, 512, 8, 2.0, dA, None, 0, None) == 1
