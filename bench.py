@@ -501,6 +501,7 @@ def run_ours(args, case):
         if not args.no_decode:
             line["quantize"] = quantize_pass(dev, max(5, args.steps // 2), args.warmup)
             line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers)
+            line["merge"] = merge_pass(dev, 5, args.warmup)
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(case)
         print(json.dumps(line), flush=True)
@@ -517,7 +518,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode-sweep GB/s measurement")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the quantize, decode-sweep and merge GB/s measurements")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode sweep (prints its JSON)")
     ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS)
     ap.add_argument("--merge-only", action="store_true", help="run only the merge + requantize pass (prints its JSON)")
