@@ -34,6 +34,9 @@ Readings adopted where the pages are silent:
   dA = s (dY B)^T X, dB = s dY^T (X A^T), no gradient for W0.
 * Merge: m = bf16(RN32(bf16(w') + s sum_j B[n, j] A[j, k])), sum and product in
   float64 with j ascending, then the NF4 + double-quant encode of m.
+* Format variants: block 64 or 128; double quantization on or off (fp32 absmax
+  per block); codes against a_b or against the dequantized scale; FP4 levels =
+  the E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by 6, both signs.
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
 tests/test_oracle_pins.py against a fact other than itself (a printed worked
@@ -235,6 +238,79 @@ def quantize_nf4_dq(w: np.ndarray) -> dict:
     q, d = double_quant(absmax)
     return {"codes": pack_codes(codes), "scales": q, "scales2": d,
             "absmax": absmax, "codes_unpacked": codes}
+
+
+# ---------------------------------------------------------------------------
+# Format variants ("QLoRA double quantization ..." page, §3.1 block size 64 or
+# 128, §3.2 the double-quantization switch, §3.3 quant type nf4 or fp4; §1.3
+# and §2.3 for the storage they cost)
+# ---------------------------------------------------------------------------
+
+def fp4_levels_f64() -> np.ndarray:
+    """FP4 levels (reading: the pages name fp4 but print no values).  The 4-bit float
+    with one sign, two exponent and one mantissa bit (E2M1) has magnitudes 0, 0.5, 1,
+    1.5, 2, 3, 4, 6; divided by 6 so that the largest is 1, both signs, ascending:
+    index 7 is -0 and index 8 is +0, so a zero normalised value takes index 7."""
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    return np.array([-m / 6.0 for m in reversed(mags)] + [m / 6.0 for m in mags], dtype=np.float64)
+
+
+def fp4_codebook() -> np.ndarray:
+    return fp4_levels_f64().astype(np.float32)
+
+
+def packed_bytes_variant(numel: int, block: int = BLOCK, dq: bool = True) -> int:
+    """4-bit codes plus the scales: u8 per block and fp32 per 256 blocks with double
+    quantization, fp32 per block without."""
+    n = int(numel)
+    nb = n // block
+    if dq:
+        return n // 2 + nb + 4 * ((nb + GROUP - 1) // GROUP)
+    return n // 2 + 4 * nb
+
+
+def quantize_variant(w: np.ndarray, block: int = BLOCK, dq: bool = True, codes_after_dq: bool = False,
+                     book: np.ndarray | None = None) -> dict:
+    """Blockwise 4-bit encode with the format's switches.
+
+    block: weights per first-level block; dq: double-quantize the block absmaxes
+    (u8 q_b + one fp32 d_g per 256 blocks) or keep them as fp32; codes_after_dq: take
+    the codes against the dequantized scale s_b = RN32(q_b d_g) instead of the absmax
+    a_b (normalised values above 1 then go to the end levels); book: the 16 levels in
+    float32, NF4 by default.  The steps are those of quantize_nf4_dq otherwise."""
+    w = np.asarray(w, np.float32).reshape(-1)
+    if w.size % block:
+        raise ValueError("numel must be a multiple of the block")
+    blocks = w.reshape(-1, block)
+    a = np.max(np.abs(blocks), axis=1)
+    out = {"absmax": a}
+    scale = a
+    if dq:
+        q, d = double_quant(a)
+        out["scales"], out["scales2"] = q, d
+        if codes_after_dq:
+            scale = dequant_scales(q, d)
+    else:
+        out["scales"] = a.copy()
+    sc = scale.astype(np.float64)[:, None]
+    safe = np.where(sc == 0.0, 1.0, sc)
+    n = (blocks.astype(np.float64) / safe).astype(np.float32)
+    n[np.broadcast_to(sc == 0.0, n.shape)] = 0.0
+    codes = nearest_code(n, book).reshape(-1)
+    out["codes"] = pack_codes(codes)
+    out["codes_unpacked"] = codes
+    return out
+
+
+def dequant_variant(codes, scales, scales2=None, block: int = BLOCK, book: np.ndarray | None = None) -> np.ndarray:
+    """w' = RN32(c[code] s_b) with s_b = RN32(q_b d_g) (scales2 given) or the fp32
+    absmax itself (double quantization off)."""
+    c = unpack_codes(codes)
+    s = dequant_scales(scales, scales2) if scales2 is not None else np.asarray(scales, np.float32)
+    if book is None:
+        book = nf4_codebook()
+    vals = book.astype(np.float64)[c].reshape(-1, block) * s.astype(np.float64)[:, None]
+    return vals.astype(np.float32).reshape(-1)
 
 
 def dequant_scales(q: np.ndarray, d: np.ndarray) -> np.ndarray:

@@ -550,3 +550,117 @@ def test_merge_requant_round_trip_bound():
     half_gap = float(np.max(np.diff(O.nf4_codebook().astype(np.float64)))) / 2
     bound = np.repeat(a * half_gap + np.abs(a - sb), 64) * (1 + 1e-6) + 1e-30
     assert np.all(np.abs(back - m.astype(np.float64)) <= bound)
+
+
+# ------------------------------------------------------- format variants
+
+def _brute_encode(w, block, book, scale_of_block):
+    """Pure-Python blockwise encode: nearest level (first index on ties) of RN32(w / scale)."""
+    lv = [float(v) for v in book]
+    codes = []
+    for b in range(len(w) // block):
+        sc = scale_of_block(b)
+        for x in w[b * block:(b + 1) * block]:
+            n = 0.0 if sc == 0.0 else _f32_rn(float(x) / sc)
+            best, bd = 0, abs(n - lv[0])
+            for k in range(1, 16):
+                dk = abs(n - lv[k])
+                if dk < bd:
+                    best, bd = k, dk
+            codes.append(best)
+    return codes
+
+
+def test_variant_defaults_reduce_to_the_nf4_dq_encode():
+    w = (np.random.default_rng(81).standard_normal(16384 * 2 + 640) * 0.02).astype(np.float32)
+    a, b = O.quantize_variant(w), O.quantize_nf4_dq(w)
+    for key in ("codes", "scales", "scales2"):
+        assert np.array_equal(a[key], b[key])
+    assert np.array_equal(O.dequant_variant(a["codes"], a["scales"], a["scales2"]),
+                          O.dequant(b["codes"], b["scales"], b["scales2"]))
+
+
+@pytest.mark.parametrize("block,dq", [(128, True), (128, False), (64, False)])
+def test_variant_encode_brute_force_python(block, dq):
+    w = (np.random.default_rng(82).standard_normal(block * 6) * 0.02).astype(np.float32)
+    w[: block] = 0.0                       # an all-zero block
+    got = O.quantize_variant(w, block=block, dq=dq)
+    absmax = [max(abs(float(x)) for x in w[b * block:(b + 1) * block]) for b in range(6)]
+    want = _brute_encode(w.tolist(), block, O.nf4_codebook(), lambda b: absmax[b])
+    assert got["codes_unpacked"].tolist() == want
+    if not dq:
+        assert got["scales"].tolist() == [np.float32(a) for a in absmax]
+
+
+def test_codes_after_dq_brute_force_python():
+    w = (np.random.default_rng(83).standard_normal(64 * 300) * 0.02).astype(np.float32)
+    got = O.quantize_variant(w, codes_after_dq=True)
+    q, d = got["scales"], got["scales2"]
+    sb = [_f32_rn(float(q[b]) * float(d[b // 256])) for b in range(300)]
+    want = _brute_encode(w.tolist(), 64, O.nf4_codebook(), lambda b: sb[b])
+    assert got["codes_unpacked"].tolist() == want
+    # the same scales as the default encode; only codes near a threshold move
+    base = O.quantize_nf4_dq(w)
+    assert np.array_equal(q, base["scales"]) and np.array_equal(d, base["scales2"])
+    moved = np.mean(got["codes_unpacked"] != base["codes_unpacked"])
+    assert 0 < moved < 0.1
+
+
+def test_variant_dq_off_round_trip_exact_on_representable_weights():
+    # w = c_k * a with a power-of-two absmax: fp32 absmax kept exactly, codes exact
+    rng = np.random.default_rng(84)
+    book = O.nf4_codebook()
+    for block in (64, 128):
+        codes = rng.integers(0, 16, size=block * 8).astype(np.uint8)
+        codes[::block] = 15                 # the absmax element of each block is +1 * a
+        a = (2.0 ** rng.integers(-12, -2, size=8)).astype(np.float32)
+        w = (book[codes].reshape(-1, block).astype(np.float64) * a[:, None]).astype(np.float32).reshape(-1)
+        got = O.quantize_variant(w, block=block, dq=False)
+        assert np.array_equal(got["codes_unpacked"], codes)
+        assert np.array_equal(O.dequant_variant(got["codes"], got["scales"], None, block=block), w)
+
+
+def test_variant_storage_closed_forms():
+    n = 4096 * 11008
+    for block, dq in ((64, True), (128, True), (64, False), (128, False)):
+        assert O.packed_bytes_variant(n, block, dq) * 8 == pytest.approx(
+            n * (4 + O.constant_bits_per_param(block=block, dq=dq)), rel=1e-6)
+    assert O.packed_bytes_variant(n) == O.packed_bytes(n)
+    # halving the block doubles the constants; DQ off costs 32/64 = 0.5 bit per weight at 64
+    assert O.constant_bits_per_param(block=64, dq=False) == 0.5
+    assert O.constant_bits_per_param(block=128, dq=False) == 0.25
+
+
+def test_fp4_table_invariants():
+    book = O.fp4_codebook()
+    assert book.size == 16 and np.all(np.diff(book.astype(np.float64)) >= 0)
+    assert book[0] == -1.0 and book[15] == 1.0 and book[7] == 0.0 and book[8] == 0.0
+    assert np.signbit(book[7]) and not np.signbit(book[8])
+    assert np.array_equal(book[::-1], -book)
+    # every level times 6 is an E2M1 magnitude: 0, 0.5, 1, 1.5, 2, 3, 4, 6
+    assert sorted({abs(float(v)) * 6 for v in O.fp4_levels_f64()}) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    # a zero normalised value takes the lower of the two zeros
+    assert int(O.nearest_code(np.zeros(1, np.float32), book)[0]) == 7
+
+
+def _rms_error(w, **kw):
+    book = kw.get("book")
+    block = kw.get("block", 64)
+    q = O.quantize_variant(w, **kw)
+    back = O.dequant_variant(q["codes"], q["scales"], q.get("scales2") if kw.get("dq", True) else None,
+                             block=block, book=book)
+    return float(np.sqrt(np.mean((back.astype(np.float64) - w.astype(np.float64)) ** 2)))
+
+
+def test_pages_claims_on_normal_weights():
+    # "QLoRA double quantization ..." page: larger blocks raise the quantization error
+    # (§3.1); double quantization barely changes it (§3.2); nf4 fits normal weights
+    # better than fp4 (§3.3)
+    w = (np.random.default_rng(85).standard_normal(16384 * 8) * 0.02).astype(np.float32)
+    e64 = _rms_error(w)
+    e128 = _rms_error(w, block=128)
+    e64_nodq = _rms_error(w, dq=False)
+    efp4 = _rms_error(w, book=O.fp4_codebook())
+    assert e128 > e64
+    assert abs(e64 - e64_nodq) < 0.02 * e64_nodq
+    assert efp4 > 1.05 * e64
