@@ -426,8 +426,8 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         cfg.blockDim = dim3(dec::kThreads);
         cfg.dynamicSmemBytes = d.smem;
         cfg.stream = st;
-        // programmatic dependent launch: the kernel builds its table and warms L2 with its
-        // frozen weights before waiting for the preceding grid
+        // programmatic dependent launch: the kernel builds its table and initialises its
+        // barriers before waiting for the preceding grid
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         at[0].val.programmaticStreamSerializationAllowed = 1;

@@ -159,7 +159,9 @@ def nearest_code(nvals: np.ndarray, book: np.ndarray | None = None) -> np.ndarra
     """Index of the nearest level for each float32 value, exact ties to the lower index.
 
     Distances are taken in float64 on the float32 inputs; np.argmin returns
-    the first minimum, which is the lower index on an exact tie.
+    the first minimum, which is the lower index on an exact tie.  Where a table
+    holds the same value twice (the FP4 table's -0 and +0), a value above it takes
+    the higher copy: the sign of a zero follows the sign of the value.
     """
     if book is None:
         book = nf4_codebook()
@@ -171,6 +173,10 @@ def nearest_code(nvals: np.ndarray, book: np.ndarray | None = None) -> np.ndarra
     for s in range(0, flat_v.size, step):
         d = np.abs(flat_v[s:s + step, None] - c[None, :])
         flat_o[s:s + step] = np.argmin(d, axis=1).astype(np.uint8)
+    dup = np.nonzero(c[1:] == c[:-1])[0]
+    for k in dup:
+        up = (flat_o == k) & (flat_v > c[k])
+        flat_o[up] = k + 1
     return out
 
 
@@ -250,9 +256,11 @@ def fp4_levels_f64() -> np.ndarray:
     """FP4 levels (reading: the pages name fp4 but print no values).  The 4-bit float
     with one sign, two exponent and one mantissa bit (E2M1) has magnitudes 0, 0.5, 1,
     1.5, 2, 3, 4, 6; divided by 6 so that the largest is 1, both signs, ascending:
-    index 7 is -0 and index 8 is +0, so a zero normalised value takes index 7."""
+    index 7 is -0 and index 8 is +0."""
     mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
     return np.array([-m / 6.0 for m in reversed(mags)] + [m / 6.0 for m in mags], dtype=np.float64)
+    # a zero normalised value takes index 7 and a positive one below 1/24 takes index 8
+    # (nearest_code: the sign of a zero follows the sign of the value)
 
 
 def fp4_codebook() -> np.ndarray:

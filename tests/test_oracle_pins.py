@@ -639,8 +639,36 @@ def test_fp4_table_invariants():
     assert np.array_equal(book[::-1], -book)
     # every level times 6 is an E2M1 magnitude: 0, 0.5, 1, 1.5, 2, 3, 4, 6
     assert sorted({abs(float(v)) * 6 for v in O.fp4_levels_f64()}) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
-    # a zero normalised value takes the lower of the two zeros
-    assert int(O.nearest_code(np.zeros(1, np.float32), book)[0]) == 7
+    # a zero normalised value takes -0, a tiny positive one +0, a tiny negative one -0
+    got = O.nearest_code(np.array([0.0, 1e-30, -1e-30, 1.0 / 24], np.float32), book).tolist()
+    assert got[:3] == [7, 8, 7]
+
+
+def test_fp4_nearest_code_matches_threshold_rule_around_every_midpoint():
+    # the threshold rule: T_k = smallest float32 strictly above the exact midpoint of
+    # levels k, k+1 (the +0 copy gets the smallest positive float32) and
+    # code = #{k : n >= T_k}; it agrees with the oracle's nearest-level rule
+    book = O.fp4_codebook()
+    lv = book.astype(np.float64)
+    T = []
+    for k in range(15):
+        mid = (lv[k] + lv[k + 1]) / 2
+        t = np.float32(mid)
+        if float(t) <= mid:
+            t = np.nextafter(t, np.float32(np.inf))
+        T.append(float(t))
+    assert all(a <= b for a, b in zip(T, T[1:]))
+    vals = []
+    for k in range(15):
+        t = np.float32(T[k])
+        for step in range(-3, 4):
+            v = t
+            for _ in range(abs(step)):
+                v = np.nextafter(v, np.float32(np.inf if step > 0 else -np.inf))
+            vals.append(v)
+    vals = np.array(vals + [0.0, -0.0, 1.0, -1.0], np.float32)
+    want = [sum(1 for t in T if float(v) >= t) for v in vals]
+    assert O.nearest_code(vals, book).tolist() == want
 
 
 def _rms_error(w, **kw):
