@@ -15,7 +15,8 @@ import torch
 
 from . import _capi
 
-__all__ = ["NF4Weight", "qlora_packed_bytes", "qlora_nf4_codebook", "qlora_quantize_nf4_dq", "qlora_dequant",
+__all__ = ["NF4Weight", "QLORA_QT_NF4", "QLORA_QT_FP4", "qlora_packed_bytes", "qlora_nf4_codebook", "qlora_codebook",
+           "qlora_quantize_nf4_dq", "qlora_dequant",
            "qlora_lora_merge_requant",
            "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
            "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
@@ -46,27 +47,32 @@ def _need(t, dtype, shape, name):
                          f"{tuple(t.shape)} on {t.device}")
 
 
+QLORA_QT_NF4, QLORA_QT_FP4 = _capi.QT_NF4, _capi.QT_FP4
+
+
 @dataclass
 class NF4Weight:
-    """Packed NF4 weight: device buffers owned by this object (codes, u8 scales, fp32 group steps)."""
+    """Packed 4-bit weight: device buffers owned by this object (codes, u8 scales, fp32 group
+    steps) and the quant type whose 16 levels the codes index (NF4 by default, or FP4)."""
     n_out: int
     n_in: int
     codes: torch.Tensor
     scales: torch.Tensor
     scales2: torch.Tensor
+    quant_type: int = QLORA_QT_NF4
 
     @classmethod
-    def empty(cls, n_out: int, n_in: int, device="cuda") -> "NF4Weight":
+    def empty(cls, n_out: int, n_in: int, device="cuda", quant_type: int = QLORA_QT_NF4) -> "NF4Weight":
         numel = n_out * n_in
         nb = numel // 64
         return cls(n_out, n_in,
                    torch.empty(numel // 2, dtype=torch.uint8, device=device),
                    torch.empty(nb, dtype=torch.uint8, device=device),
-                   torch.empty((nb + 255) // 256, dtype=torch.float32, device=device))
+                   torch.empty((nb + 255) // 256, dtype=torch.float32, device=device), int(quant_type))
 
     def c_struct(self) -> _capi.Nf4WeightC:
         return _capi.Nf4WeightC(self.n_out, self.n_in, self.codes.data_ptr(), self.scales.data_ptr(),
-                                self.scales2.data_ptr())
+                                self.scales2.data_ptr(), int(self.quant_type))
 
 
 def qlora_packed_bytes(numel: int) -> int:
@@ -76,6 +82,12 @@ def qlora_packed_bytes(numel: int) -> int:
 def qlora_nf4_codebook() -> list[float]:
     buf = (ctypes.c_float * 16)()
     _capi.check("qlora_nf4_codebook", _lib().qlora_nf4_codebook(buf))
+    return list(buf)
+
+
+def qlora_codebook(quant_type: int) -> list[float]:
+    buf = (ctypes.c_float * 16)()
+    _capi.check("qlora_codebook", _lib().qlora_codebook(int(quant_type), buf))
     return list(buf)
 
 

@@ -83,9 +83,25 @@ static double norm_ppf_as241(double p) {
 }
 
 struct Codebook {
-    float level[16];     // ascending NF4 levels, float32
+    float level[16];     // ascending levels, float32
     float thresh[16];    // thresh[k] = smallest float32 above the exact midpoint of levels k, k+1; [15] = +inf
 };
+
+// Levels rounded to float32 and the encode thresholds: a value n takes code
+// #{k : n >= thresh[k]}, the nearest level with exact ties to the lower index (two
+// equal levels, the FP4 table's -0 and +0, split by sign: the threshold between
+// them is the smallest positive float32).
+static void fill_codebook(Codebook &cb, const double (&v)[16]) {
+    for (int i = 0; i < 16; ++i) cb.level[i] = static_cast<float>(v[i]);
+    for (int k = 0; k < 15; ++k) {
+        // midpoint of two floats: exact in double
+        const double mid = (static_cast<double>(cb.level[k]) + static_cast<double>(cb.level[k + 1])) * 0.5;
+        float t = static_cast<float>(mid);
+        if (static_cast<double>(t) <= mid) t = std::nextafter(t, INFINITY);
+        cb.thresh[k] = t;
+    }
+    cb.thresh[15] = INFINITY;
+}
 
 // NF4 levels: normal quantiles at equal probability steps inside the offset
 // delta, normalised by Phi^-1(delta), 7 negative + exact 0 + 8 positive.
@@ -101,17 +117,31 @@ static const Codebook &codebook() {
         for (int j = 1; j <= 8; ++j) v[7 + j] = norm_ppf_as241(0.5 + j * (delta - 0.5) / 8.0) / top;
         v[0] = -1.0;
         v[15] = 1.0;
-        for (int i = 0; i < 16; ++i) cb.level[i] = static_cast<float>(v[i]);
-        for (int k = 0; k < 15; ++k) {
-            // midpoint of two floats: exact in double
-            const double mid = (static_cast<double>(cb.level[k]) + static_cast<double>(cb.level[k + 1])) * 0.5;
-            float t = static_cast<float>(mid);
-            if (static_cast<double>(t) <= mid) t = std::nextafter(t, INFINITY);
-            cb.thresh[k] = t;
-        }
-        cb.thresh[15] = INFINITY;
+        fill_codebook(cb, v);
     });
     return cb;
+}
+
+// FP4 levels: the E2M1 4-bit float magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by
+// 6 (largest 1), both signs, ascending; index 7 is -0 and index 8 is +0.
+static const Codebook &fp4_codebook() {
+    static Codebook cb;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const double mags[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+        double v[16];
+        for (int i = 0; i < 8; ++i) {
+            v[7 - i] = -mags[i] / 6.0;
+            v[8 + i] = mags[i] / 6.0;
+        }
+        fill_codebook(cb, v);
+    });
+    return cb;
+}
+
+// The table of a weight's 4-bit quant type (checked by check_weight).
+static const Codebook &codebook_for(int32_t quant_type) {
+    return quant_type == QLORA_QT_FP4 ? fp4_codebook() : codebook();
 }
 
 // ------------------------------------------------------------------ TMA descriptors
@@ -220,6 +250,8 @@ static qlora_status check_weight(const qlora_nf4_weight *w) {
     if (!w->codes || !w->scales || !w->scales2) return fail(QLORA_ERR_ARG, "weight buffers must be non-NULL");
     if (!aligned16(w->codes) || !aligned16(w->scales) || !aligned16(w->scales2))
         return fail(QLORA_ERR_ALIGN, "weight buffers must be 16-byte aligned");
+    if (w->quant_type != QLORA_QT_NF4 && w->quant_type != QLORA_QT_FP4)
+        return fail(QLORA_ERR_ARG, "quant_type (%d) must be QLORA_QT_NF4 (0) or QLORA_QT_FP4 (1)", w->quant_type);
     return QLORA_OK;
 }
 

@@ -2,6 +2,7 @@
 // Every kernel lives in a header of this directory; this file is the only translation unit.
 
 #include <algorithm>
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -27,9 +28,12 @@ namespace {
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-CodebookArg codebook_arg() {
+static_assert(sizeof(qlora_nf4_weight) == 48 && offsetof(qlora_nf4_weight, quant_type) == 40,
+              "the weight descriptor layout is part of the ABI");
+
+CodebookArg codebook_arg(int32_t quant_type) {
     CodebookArg a;
-    const Codebook &cb = codebook();
+    const Codebook &cb = codebook_for(quant_type);
     for (int i = 0; i < 16; ++i) {
         a.level[i] = cb.level[i];
         a.thresh[i] = cb.thresh[i];
@@ -305,6 +309,15 @@ qlora_status qlora_nf4_codebook(float out[16]) {
     return QLORA_OK;
 }
 
+qlora_status qlora_codebook(int quant_type, float *out) {
+    if (!out) return fail(QLORA_ERR_ARG, "out is NULL");
+    if (quant_type != QLORA_QT_NF4 && quant_type != QLORA_QT_FP4)
+        return fail(QLORA_ERR_ARG, "quant_type (%d) must be QLORA_QT_NF4 (0) or QLORA_QT_FP4 (1)", quant_type);
+    const Codebook &cb = codebook_for(quant_type);
+    for (int i = 0; i < 16; ++i) out[i] = cb.level[i];
+    return QLORA_OK;
+}
+
 const char *qlora_last_error(void) { return t_last_error; }
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
@@ -336,7 +349,7 @@ qlora_status qlora_quantize_nf4_dq(const float *W, const qlora_nf4_weight *w, vo
     const int64_t ngroups = ceil_div(nblocks, 256);
     if (ngroups > INT32_MAX) return fail(QLORA_ERR_SHAPE, "weight too large");
     nf4_encode_dq_kernel<<<static_cast<unsigned>(ngroups), kEncThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        W, w->codes, w->scales, w->scales2, nblocks, codebook_arg());
+        W, w->codes, w->scales, w->scales2, nblocks, codebook_arg(w->quant_type));
     return launch_check("nf4_encode_dq_kernel launch");
 }
 
@@ -351,10 +364,10 @@ qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (out_is_bf16)
         nf4_dequant_kernel<true><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, w->scales, w->scales2, out,
-                                                                               n8, codebook_arg());
+                                                                               n8, codebook_arg(w->quant_type));
     else
         nf4_dequant_kernel<false><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, w->scales, w->scales2, out,
-                                                                                n8, codebook_arg());
+                                                                                n8, codebook_arg(w->quant_type));
     return launch_check("nf4_dequant_kernel launch");
 }
 
@@ -375,7 +388,7 @@ qlora_status qlora_lora_merge_requant(const qlora_nf4_weight *w_in, const qlora_
     nf4_lora_merge_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
         w_in->codes, w_in->scales, w_in->scales2, r > 0 ? reinterpret_cast<const uint16_t *>(A) : nullptr,
         r > 0 ? reinterpret_cast<const uint16_t *>(B) : nullptr, r, r > 0 ? scaling : 0.f, w_in->n_out, w_in->n_in,
-        W_scratch, codebook_arg());
+        W_scratch, codebook_arg(w_in->quant_type));
     QL_TRY(launch_check("nf4_lora_merge_kernel launch"));
     return qlora_quantize_nf4_dq(W_scratch, w_out, stream);
 }
@@ -410,7 +423,7 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         p.r = r;
         p.units = static_cast<int>(ceil_div(N, dec::kRows));
         p.scaling = scaling;
-        const Codebook &cbd = codebook();
+        const Codebook &cbd = codebook_for(w->quant_type);
         for (int i = 0; i < 16; ++i) p.level[i] = cbd.level[i];
         // codes as u8 [N, K/2] in [32 rows x 128 B] boxes (3-D: four 256-k chunks per box);
         // X and A as [K/64][rows][64] bf16 chunks, sixteen chunks per box
@@ -457,7 +470,7 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         QL_TRY(launch_skinny(X, 0, A, 0, K, M, r, 1.0f, uacc, r, 1, st));
         QL_TRY(launch_finalize(uacc, M * r, scaling, U_save, us, st));
     }
-    const Codebook &cb = codebook();
+    const Codebook &cb = codebook_for(w->quant_type);
 
     if (pair) {
         const int BN = pair_token_tile(M);
@@ -573,7 +586,7 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
         QL_TRY(launch_skinny(dY, 0, B, 1, N, M, r, 1.0f, gacc, r, 1, st));
         QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
     }
-    const Codebook &cb = codebook();
+    const Codebook &cb = codebook_for(w->quant_type);
 
     if (pair) {
         const int BN = pair_token_tile(M);

@@ -59,12 +59,24 @@ typedef enum {
     QLORA_ERR_UNSUPPORTED = 7 /* no sm_100 device / wrong architecture           */
 } qlora_status;
 
-/* Packed NF4 + double-quant weight.  All three buffers are device memory
+/* 4-bit level sets ("QLoRA double quantization ..." page, section 3.3: the
+ * quant type is nf4 or fp4).  NF4: the normal-quantile levels of
+ * qlora_nf4_codebook.  FP4 (a reading; the pages print no values): the E2M1
+ * 4-bit float magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by 6, both signs,
+ * ascending, with -0 at index 7 and +0 at index 8; a zero or tiny negative
+ * normalised value takes index 7, a tiny positive one index 8. */
+enum { QLORA_QT_NF4 = 0, QLORA_QT_FP4 = 1 };
+
+/* Packed 4-bit + double-quant weight.  All three buffers are device memory
  * owned by the caller.  numel = n_out * n_in must be a multiple of 64 and
  * n_in must be a multiple of 64 (blocks never straddle rows).
+ * quant_type selects the 16 levels (QLORA_QT_NF4 or QLORA_QT_FP4); every call
+ * encodes, dequantizes and multiplies with the levels of the weight's type.
+ * The descriptor is 48 bytes (the int32 quant_type is followed by padding).
  *   codes   : numel / 2 bytes; weight element 2j (row-major flattening) is
  *             in bits 0-3 of byte j, element 2j+1 in bits 4-7; each code
- *             indexes the 16-entry NF4 codebook (see qlora_nf4_codebook).
+ *             indexes the 16 levels of the weight's quant type (see
+ *             qlora_codebook).
  *   scales  : numel / 64 bytes; block b (elements [64b, 64b+64)) has first
  *             level scale q_b in 0..255.
  *   scales2 : ceil(numel / 16384) floats; group g (blocks [256g, 256g+256))
@@ -76,6 +88,7 @@ typedef struct {
     uint8_t *codes;
     uint8_t *scales;
     float *scales2;
+    int32_t quant_type;
 } qlora_nf4_weight;
 
 /* Bytes of the three packed buffers together: numel/2 + numel/64 +
@@ -90,6 +103,11 @@ size_t qlora_packed_bytes(int64_t numel);
  * delta = ((1 - 1/30) + (1 - 1/32)) / 2, each divided by Phi^-1(delta),
  * plus an exact zero.  Returns QLORA_ERR_ARG if out is NULL. */
 qlora_status qlora_nf4_codebook(float out[16]);
+
+/* The 16 levels of quant type `quant_type` (QLORA_QT_NF4 or QLORA_QT_FP4) as
+ * float32, ascending, into the HOST array out.  QLORA_ERR_ARG for another
+ * type or a NULL out. */
+qlora_status qlora_codebook(int quant_type, float *out);
 
 /* Encode: W [n_out, n_in] fp32 (device) -> w->codes, w->scales, w->scales2.
  * Per block of 64: a_b = max |w|; code = index of the nearest level to

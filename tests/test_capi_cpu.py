@@ -112,6 +112,26 @@ def test_validation_rejects_before_launch(lib):
     assert lib.qlora_lora_grad_AB(X, Y, A, B, 16, 256, 512, 8, 2.0, dA, dB, 3, None) == 1
 
 
+def test_weight_descriptor_layout_and_quant_type(lib):
+    # the C side pins the same layout with a static_assert
+    assert ctypes.sizeof(_capi.Nf4WeightC) == 48 and _capi.Nf4WeightC.quant_type.offset == 40
+    w = _w()
+    w.quant_type = 2
+    assert lib.qlora_dequant(ctypes.byref(w), ctypes.c_void_p(0x4000), 0, None) == 1
+    assert "quant_type" in _err(lib)
+    assert lib.qlora_quantize_nf4_dq(ctypes.c_void_p(0x4000), ctypes.byref(w), None) == 1
+
+
+def test_codebooks_match_oracle_bit_for_bit(lib):
+    for qt, book in ((0, O.nf4_codebook()), (1, O.fp4_codebook())):
+        buf = (ctypes.c_float * 16)()
+        assert lib.qlora_codebook(qt, buf) == 0
+        assert np.array_equal(np.array(list(buf), np.float32).view(np.uint32), book.view(np.uint32))
+    buf = (ctypes.c_float * 16)()
+    assert lib.qlora_codebook(2, buf) == 1
+    assert lib.qlora_codebook(0, None) == 1
+
+
 def test_binding_refuses_missing_library(tmp_path):
     saved = _capi._lib
     try:
