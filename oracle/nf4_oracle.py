@@ -37,6 +37,8 @@ Readings adopted where the pages are silent:
 * Format variants: block 64 or 128; double quantization on or off (fp32 absmax
   per block); codes against a_b or against the dequantized scale; FP4 levels =
   the E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 divided by 6, both signs.
+* Q8_0: blocks of 32, d = fp16(max|w| / 127), q = clamp(rint_even(w / d), -127,
+  127), w' = q d.
 
 Parity status: every function here is pinned by a ``-m "not gpu"`` test in
 tests/test_oracle_pins.py against a fact other than itself (a printed worked
@@ -319,6 +321,43 @@ def dequant_variant(codes, scales, scales2=None, block: int = BLOCK, book: np.nd
         book = nf4_codebook()
     vals = book.astype(np.float64)[c].reshape(-1, block) * s.astype(np.float64)[:, None]
     return vals.astype(np.float32).reshape(-1)
+
+
+# ---------------------------------------------------------------------------
+# Q8_0 block format ("Training LoRA directly on GGUF quantized weights" page,
+# §1.1: 32 weights share one fp16 scale, a little over one byte per weight;
+# §2.2: blockwise dequant inside the GEMM or a one-shot dequant to bf16).
+# Reading: symmetric int8 per block as in the "Quantized vs. non-quantized
+# weights" page, §2.1: d = fp16(max|w| / 127), q = clamp(rint_even(w / d),
+# -127, 127), w' = q * d; a block of zeros has d = 0 and q = 0.
+# ---------------------------------------------------------------------------
+
+Q8_BLOCK = 32
+
+
+def q8_0_packed_bytes(numel: int) -> int:
+    """32 int8 values plus one fp16 scale per block: 34 bytes per 32 weights."""
+    return (int(numel) // Q8_BLOCK) * (Q8_BLOCK + 2)
+
+
+def quantize_q8_0(w: np.ndarray) -> dict:
+    """Blockwise symmetric int8: the fp16 scale of each block of 32 and the int8 values."""
+    w = np.asarray(w, np.float32).reshape(-1)
+    if w.size % Q8_BLOCK:
+        raise ValueError("numel must be a multiple of 32")
+    blocks = w.reshape(-1, Q8_BLOCK).astype(np.float64)
+    d = (np.max(np.abs(blocks), axis=1) / 127.0).astype(np.float16)
+    d64 = d.astype(np.float64)[:, None]
+    safe = np.where(d64 == 0.0, 1.0, d64)
+    q = np.clip(np.rint(blocks / safe), -127, 127)
+    q[np.broadcast_to(d64 == 0.0, q.shape)] = 0
+    return {"q": q.astype(np.int8).reshape(-1), "d": d}
+
+
+def dequant_q8_0(q: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """w' = q * d, exact in float32 (an 8-bit integer times an 11-bit fp16 significand)."""
+    qb = np.asarray(q, np.int8).reshape(-1, Q8_BLOCK).astype(np.float64)
+    return (qb * np.asarray(d, np.float16).astype(np.float64)[:, None]).astype(np.float32).reshape(-1)
 
 
 def dequant_scales(q: np.ndarray, d: np.ndarray) -> np.ndarray:

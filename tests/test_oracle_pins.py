@@ -692,3 +692,53 @@ def test_pages_claims_on_normal_weights():
     assert e128 > e64
     assert abs(e64 - e64_nodq) < 0.02 * e64_nodq
     assert efp4 > 1.05 * e64
+
+
+# ------------------------------------------------------------------- Q8_0
+
+def test_q8_0_storage_matches_the_page_figures():
+    # GGUF page §1.1: a little over one byte per weight; a 3.8B model of 7.6 GB in bf16
+    # is about 4 GB in Q8_0
+    n = 3_800_000_000 // 32 * 32
+    assert O.q8_0_packed_bytes(n) / n == 34 / 32
+    assert 2 * n / 1e9 == pytest.approx(7.6, abs=0.01)
+    assert O.q8_0_packed_bytes(n) / 1e9 == pytest.approx(4.0, abs=0.05)
+
+
+def test_q8_0_brute_force_python():
+    rng = np.random.default_rng(91)
+    w = (rng.standard_normal(32 * 20) * 0.02).astype(np.float32)
+    w[:32] = 0.0
+    got = O.quantize_q8_0(w)
+    for b in range(20):
+        blk = [float(x) for x in w[b * 32:(b + 1) * 32]]
+        d = float(np.float16(max(abs(x) for x in blk) / 127.0))
+        assert float(got["d"][b]) == d
+        for i, x in enumerate(blk):
+            if d == 0.0:
+                want = 0
+            else:
+                t = x / d
+                fl = math.floor(t)
+                frac = t - fl
+                want = fl + (1 if frac > 0.5 or (frac == 0.5 and fl % 2 == 1) else 0)
+                want = max(-127, min(127, want))
+            assert int(got["q"][b * 32 + i]) == want
+
+
+def test_q8_0_round_trip_bound_and_exact_values():
+    rng = np.random.default_rng(92)
+    w = (rng.standard_normal(32 * 512) * 0.02).astype(np.float32)
+    g = O.quantize_q8_0(w)
+    back = O.dequant_q8_0(g["q"], g["d"]).astype(np.float64)
+    d = np.repeat(g["d"].astype(np.float64), 32)
+    # half a step, plus the clamp at 127 when fp16 rounded the scale down
+    assert np.all(np.abs(back - w) <= d * 0.5 + np.abs(w) * 2.0 ** -10 + 1e-30)
+    # integers times a representable scale come back exactly
+    d0 = np.float16(2.0 ** -9)
+    q0 = rng.integers(-127, 128, size=32 * 8)
+    q0[::32] = 127
+    w0 = (q0.astype(np.float64) * float(d0)).astype(np.float32)
+    g0 = O.quantize_q8_0(w0)
+    assert np.array_equal(g0["q"].astype(np.int64), q0) and np.all(g0["d"] == d0)
+    assert np.array_equal(O.dequant_q8_0(g0["q"], g0["d"]), w0)
