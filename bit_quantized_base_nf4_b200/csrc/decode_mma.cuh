@@ -267,6 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // -------------------------------------------------------------------- consumers
+    // A wait that times out sets the CTA's abort flag and the device error word (which
+    // the host reports); the consumers then run on without waiting, so that all eight
+    // warps still reach every named barrier and the CTA exits.
     const int pr = warp & 3, gs = warp >> 2;
     const int g = lane >> 2, t = lane & 3;
     const int sg = ((g & 1) << 2) | (g >> 1);          // W row (in its n8 group) of MMA column g
