@@ -228,15 +228,17 @@ DECODE_MS = (1, 4, 16)
 DECODE_R, DECODE_ALPHA = 8, 16.0
 
 
-def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS):
+def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS, with_gate=False, ms=DECODE_MS):
     """Forward over the 32-layer 7B weight set (Q, K, V, O 4096x4096, up 11008x4096, down
     4096x11008; LoRA r=8 on Q/K/V/O) at M = 1, 4, 16 tokens, one library call per matrix,
     captured once in a CUDA graph per M.  Calls carry no data dependency on each other.
-    Returns algorithmic GB/s = (packed weights + X + Y + LoRA A/B bytes) / sweep time."""
+    with_gate adds a gate projection (11008x4096) per layer: 6.48e9 weights, the count the
+    decode configuration quotes.  Returns algorithmic GB/s = (packed weights + X + Y + LoRA
+    A/B bytes) / sweep time."""
     import torch
     import bit_quantized_base_nf4_b200 as q
     from bit_quantized_base_nf4_b200 import synthetic as syn
-    shapes = syn.decode_layer_shapes()
+    shapes = syn.decode_layer_shapes(with_gate)
     r, s = DECODE_R, DECODE_ALPHA / DECODE_R
     mats = []
     for layer in range(layers):
@@ -253,7 +255,7 @@ def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS):
     q.qlora_sync_status()
     widths = sorted({K for _, _, K, _, _ in mats} | {N for _, N, _, _, _ in mats})
     out = {}
-    for M in DECODE_MS:
+    for M in ms:
         X = {K: syn.decode_inputs(M, K, 4900 + K).to(dev) for K in widths}
         Y = {N: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for N in widths}
         ws = torch.empty(max(q.qlora_workspace_bytes(M, N, K, r) for _, N, K, _, _ in mats), dtype=torch.uint8,
@@ -289,7 +291,8 @@ def decode_sweep(dev, steps, warmup, layers=DECODE_LAYERS):
         out[f"M={M}"] = {"GB/s": gbs, "ms_per_sweep": ms, "bytes_per_sweep": nbytes,
                          "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
         del g
-    out["workload"] = (f"7B decode sweep: {layers} layers x {{Q,K,V,O 4096x4096, up 11008x4096, down 4096x11008}} = "
+    gate = " gate 11008x4096," if with_gate else ""
+    out["workload"] = (f"7B decode sweep: {layers} layers x {{Q,K,V,O 4096x4096,{gate} up 11008x4096, down 4096x11008}} = "
                        f"{sum(N * K for _, N, K, _, _ in mats):.3e} NF4 weights, LoRA r=8 on Q/K/V/O; "
                        "one forward call per matrix, no inter-call dependency, CUDA graph per M; "
                        "working set >> L2 (no flush)")
@@ -501,6 +504,9 @@ def run_ours(args, case):
         if not args.no_decode:
             line["quantize"] = quantize_pass(dev, max(5, args.steps // 2), args.warmup)
             line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers)
+            # the configuration's "~6.5e9 weights" counts a gate projection per layer as well
+            line["decode_with_gate"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers,
+                                                    with_gate=True, ms=(1,))
             line["merge"] = merge_pass(dev, 5, args.warmup)
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(case)
