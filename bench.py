@@ -371,6 +371,15 @@ def merge_pass(dev, steps, warmup):
     return out
 
 
+def _side_leg(fn):
+    """Runs a measurement beside the headline step; a failure is reported in its key
+    instead of losing the whole JSON line."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001 - any failure of a side measurement is reported, not raised
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
 # ----------------------------------------------------------------------------- CUDA leg
 
 def run_ours(args, case):
@@ -502,14 +511,15 @@ def run_ours(args, case):
                         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         if not args.no_decode:
-            line["quantize"] = quantize_pass(dev, max(5, args.steps // 2), args.warmup)
-            line["decode"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers)
+            k = max(5, args.steps // 2)
+            line["quantize"] = _side_leg(lambda: quantize_pass(dev, k, args.warmup))
+            line["decode"] = _side_leg(lambda: decode_sweep(dev, k, args.warmup, args.decode_layers))
             # the configuration's "~6.5e9 weights" counts a gate projection per layer as well
-            line["decode_with_gate"] = decode_sweep(dev, max(5, args.steps // 2), args.warmup, args.decode_layers,
-                                                    with_gate=True, ms=(1,))
-            line["merge"] = merge_pass(dev, 5, args.warmup)
+            line["decode_with_gate"] = _side_leg(lambda: decode_sweep(dev, k, args.warmup, args.decode_layers,
+                                                                      with_gate=True, ms=(1,)))
+            line["merge"] = _side_leg(lambda: merge_pass(dev, 5, args.warmup))
         if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(case)
+            line["cpu_baseline"] = _side_leg(lambda: cpu_baseline(case))
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
