@@ -20,7 +20,7 @@ __all__ = ["NF4Weight", "QLORA_QT_NF4", "QLORA_QT_FP4", "qlora_packed_bytes", "q
            "qlora_lora_merge_requant",
            "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
            "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
-           "qlora_sync_status", "QloraError"]
+           "qlora_sync_status", "qlora_set_wait_limit_ns", "qlora_probe_wait_timeout", "QloraError"]
 
 QloraError = _capi.QloraError
 
@@ -195,3 +195,13 @@ def qlora_lora_grad_AB(X, dY, U, G, r: int, scaling: float, dA, dB, accumulate: 
 
 def qlora_sync_status(stream=None) -> None:
     _capi.check("qlora_sync_status", _lib().qlora_sync_status(_stream(stream)))
+
+
+def qlora_set_wait_limit_ns(ns: int) -> None:
+    """Time after which a kernel pipeline wait gives up on the current device (default 2e9 ns)."""
+    _capi.check("qlora_set_wait_limit_ns", _lib().qlora_set_wait_limit_ns(int(ns)))
+
+
+def qlora_probe_wait_timeout(stream=None) -> None:
+    """Enqueue the self-test kernel whose wait runs out; the next sync reports QLORA_ERR_TIMEOUT."""
+    _capi.check("qlora_probe_wait_timeout", _lib().qlora_probe_wait_timeout(_stream(stream)))

@@ -41,6 +41,8 @@ SIGNATURES = {
     "qlora_lora_grad_AB": (_int, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _f32, _vp, _vp, _int, _vp]),
     "qlora_sync_status": (_int, [_vp]),
     "qlora_last_error": (ctypes.c_char_p, []),
+    "qlora_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
+    "qlora_probe_wait_timeout": (_int, [_vp]),
 }
 
 _lib = None

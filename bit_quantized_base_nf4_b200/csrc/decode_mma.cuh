@@ -375,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t word = cwv[jj >> 1];
                         const uint32_t sh = 16 * (jj & 1);
                         const uint32_t e0 = (word >> sh) & 0xFFu, e1 = (word >> (sh + 8)) & 0xFFu;
-                        const uint32_t b0 = bf16x2_mul(lds32(lut + (e0 << 7)), sc[gg]);
-                        const uint32_t b1 = bf16x2_mul(lds32(lut + (e1 << 7)), sc[gg]);
+                        const uint32_t b0 = bf16x2_mul(lds32_const(lut + (e0 << 7)), sc[gg]);
+                        const uint32_t b1 = bf16x2_mul(lds32_const(lut + (e1 << 7)), sc[gg]);
                         mma_bf16_16816(acc[gg][jj & 1], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, b0, b1);
                     }
                 }

@@ -25,7 +25,9 @@
 //                        swizzled into A slot s % 4, then arrives on a_full
 //   MMA (warp 1, even)   four tcgen05.mma (K = 16), A and B from shared memory
 // Commits are multicast to both CTAs (free, acc_full); each CTA then reads back
-// its own 128 x BN accumulator and writes dX.
+// its own 128 x BN accumulator and writes dX, or, when the contraction over n is
+// split across blockIdx.z (few output tiles: small M), adds it into an fp32
+// accumulator that a finalize kernel rounds to bf16.
 #pragma once
 
 #include <cstdint>
@@ -51,8 +53,10 @@ struct Params {
     const uint8_t *scales;
     const float *scales2;
     const uint16_t *Alora;   // [r, K] bf16 or nullptr
-    uint16_t *dX;            // [M, K] bf16
+    uint16_t *dX;            // [M, K] bf16 (one split)
+    float *dXacc;            // [M, K] fp32 accumulator, zeroed by the host (several splits), or nullptr
     int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
+    int nb_per_split;        // 64-n stages per split along blockIdx.z (a multiple of 4)
     float level[16];
 };
 
@@ -89,8 +93,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int m0 = blockIdx.y * p.BN;
     const int my_m0 = m0 + int(rank) * half_bn;
     const int KB = p.K / 64;
-    const int NB = (p.N + 63) / 64;               // main stages (64 n each)
-    const int LS = p.r > 0 ? (p.r + 63) / 64 : 0; // adapter stages (64 j each)
+    const int NB_all = (p.N + 63) / 64;
+    const int nb_begin = blockIdx.z * p.nb_per_split;          // first 64-n stage of this split
+    const int NB = min(NB_all, nb_begin + p.nb_per_split) - nb_begin;   // main stages (64 n each)
+    // adapter stages (64 j each), on the last split only
+    const int LS = (p.r > 0 && nb_begin + NB == NB_all) ? (p.r + 63) / 64 : 0;
     const int total = NB + LS;
     const int nchunk = (NB + 3) / 4;
     const uint32_t ncols = tmem_cols(p.BN);
@@ -142,7 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t bar0 = mapa_shared(smem_u32(&y_full[sx]), 0);
                 if (rank == 0) mbar_arrive_expect_tx(&y_full[sx], 2 * ysb);
                 if (s < NB)
-                    tma_load_2d_pair(sY + sx * ysb, &tmY, bar0, s * 64, my_m0);
+                    tma_load_2d_pair(sY + sx * ysb, &tmY, bar0, (nb_begin + s) * 64, my_m0);
                 else
                     tma_load_2d_pair(sY + sx * ysb, &tmG, bar0, (s - NB) * 64, my_m0);
                 issued = s + 1;
@@ -163,8 +170,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int sc = c % SC;
                 if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(&c_full[sc], kCodeChunkBytes);
-                // rows n = 256c .., bytes k0/2 .. k0/2 + 63
-                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], k0 / 2, c * kChunkRows);
+                // rows n = 64 nb_begin + 256c .., bytes k0/2 .. k0/2 + 63
+                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], k0 / 2, nb_begin * 64 + c * kChunkRows);
                 issued = c + 1;
             }
             for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
@@ -208,7 +215,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         bool ok = true;
 
         auto load_scale = [&](int s, uint32_t &qv, float &dv) {
-            const int n = s * 64 + nl;
+            const int n = (nb_begin + s) * 64 + nl;
             qv = 0;
             dv = 0.f;
             if (kvalid && s < NB && n < p.N) {
@@ -246,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int by = 0; by < 4; ++by) {
                         const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
-                        out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                        out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
                     }
                 }
             } else {
@@ -291,12 +298,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_wait_ld16(v);
                 if (k < p.K) {
                     const int mb = m0 + ch * 16;
+                    if (p.dXacc) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (mb + i < p.M) {
-                            __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
-                            p.dX[int64_t(mb + i) * p.K + k] = *reinterpret_cast<uint16_t *>(&hv);
-                        }
+                        for (int i = 0; i < 16; ++i)
+                            if (mb + i < p.M) atomicAdd(p.dXacc + int64_t(mb + i) * p.K + k, __uint_as_float(v[i]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (mb + i < p.M) {
+                                __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
+                                p.dX[int64_t(mb + i) * p.K + k] = *reinterpret_cast<uint16_t *>(&hv);
+                            }
+                    }
                 }
             }
         }

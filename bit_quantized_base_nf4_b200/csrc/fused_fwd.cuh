@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int by = 0; by < 4; ++by) {
                         const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
-                        out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                        out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
                     }
                 }
             } else {

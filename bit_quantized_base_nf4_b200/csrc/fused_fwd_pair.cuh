@@ -253,7 +253,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int by = 0; by < 4; ++by) {
                             const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
-                            out[w8 * 4 + by] = bf16x2_mul(lds32(lut + (e << 7)), s2);
+                            out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
                         }
                     }
                     tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);

@@ -12,8 +12,10 @@ namespace qlora {
 __device__ int g_device_error = 0;
 constexpr int kDeviceErrTimeout = 6;
 constexpr int kDeviceErrTmemStore = 7;   // a TMEM store did not read back as written
-// Time after which a single pipeline wait gives up (ns of %globaltimer).
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Time after which a single pipeline wait gives up (ns of %globaltimer); 2 s unless
+// changed by qlora_set_wait_limit_ns.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -54,7 +56,7 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t *bar, uint32_t parity
 
 // Waits until the phase of `bar` with parity `parity` has completed.  Returns
 // false (after raising the CTA's abort flag and the device error word) if the
-// wait exceeds kWaitLimitNs or another role of the CTA has already aborted.
+// wait exceeds g_wait_limit_ns or another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -62,7 +64,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > g_wait_limit_ns) {
                 *abort_flag = 1;
                 atomicExch(&g_device_error, kDeviceErrTimeout);
                 return false;
@@ -239,17 +241,30 @@ __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&v)[16]) {
 }
 
 // ------------------------------------------------------------------ shared-memory helpers
+// Shared-memory loads of data that barriers guard (code tiles): the "memory"
+// clobber keeps the compiler from moving them across the barrier operations or
+// other memory accesses around them.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
     return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
     uint2 v;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
     return v;
 }
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+// Load from a table that is written once before the CTA's first __syncthreads and
+// only read afterwards (the code -> level tables); no ordering constraint needed.
+__device__ __forceinline__ uint32_t lds32_const(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
@@ -308,7 +323,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((it & 31u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > g_wait_limit_ns) {
                 *abort_flag = 1;
                 atomicExch(&g_device_error, kDeviceErrTimeout);
                 return false;

@@ -12,7 +12,6 @@
 #include "skinny_mma.cuh"
 #include "fused_fwd.cuh"
 #include "fused_fwd_pair.cuh"
-#include "fused_bwd.cuh"
 #include "fused_bwd_pair.cuh"
 #include "decode_mma.cuh"
 
@@ -22,6 +21,21 @@ using namespace qlora;
 // memory on every device where the module is loaded; zero-filled at load, and
 // each call clears the parts it accumulates into.
 static __device__ __align__(256) uint8_t g_static_scratch[QLORA_STATIC_SCRATCH_BYTES];
+
+// Self-test of the bounded-wait path: one thread waits on a barrier that nothing
+// arrives on, with the same wait every pipeline uses; it gives up after the
+// current limit, raises the device error word and returns.
+__global__ void wait_probe_kernel() {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag);
+}
 
 namespace {
 
@@ -180,9 +194,31 @@ size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
     const bool split = !use_pair_fwd(M) && plan_gemm(M, N, K / 64).splits > 1;
     return ws_layout(M, N, r, split).total;
 }
+// dX plan: CTA pairs (256 k columns x BN tokens per pair) at every M.  When the pair
+// tiles would fill less than half of the SM pairs (small M), the contraction over n
+// is split along blockIdx.z into whole four-stage code chunks, and the splits add
+// into an fp32 accumulator.
+struct DxPlan {
+    int BN;
+    int64_t pairs, tiles_tok;
+    int splits, nb_per_split;
+};
+DxPlan plan_dx(int64_t M, int64_t N, int64_t K) {
+    DxPlan d;
+    d.BN = pair_token_tile(M);
+    d.pairs = ceil_div(K, 2 * bwdp::BM);
+    d.tiles_tok = ceil_div(M, d.BN);
+    const int64_t nb = ceil_div(N, 64);
+    const int64_t tiles = d.pairs * d.tiles_tok;
+    const int64_t pair_slots = std::max(1, sm_count() / 2);
+    int64_t splits = 1;
+    if (tiles * 2 <= pair_slots) splits = std::min(ceil_div(pair_slots, tiles), std::max<int64_t>(1, nb / 4));
+    d.nb_per_split = static_cast<int>(ceil_div(ceil_div(nb, splits), 4) * 4);
+    d.splits = static_cast<int>(ceil_div(nb, d.nb_per_split));
+    return d;
+}
 size_t bwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    const bool split = !use_pair_fwd(M) && plan_gemm(M, K, ceil_div(N, 64)).splits > 1;
-    return ws_layout(M, K, r, split).total;
+    return ws_layout(M, K, r, plan_dx(M, N, K).splits > 1).total;
 }
 
 // Launches the rank-r tensor-core product out[i*ld_i + j*ld_j] += scaling *
@@ -319,6 +355,20 @@ qlora_status qlora_codebook(int quant_type, float *out) {
 }
 
 const char *qlora_last_error(void) { return t_last_error; }
+
+qlora_status qlora_set_wait_limit_ns(uint64_t ns) {
+    if (ns < 1000000ull || ns > 60000000000ull)
+        return fail(QLORA_ERR_ARG, "wait limit %llu ns outside [1e6, 6e10]", (unsigned long long)ns);
+    QL_TRY(require_sm100());
+    const unsigned long long v = ns;
+    return cuda_check(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)), "set the wait limit");
+}
+
+qlora_status qlora_probe_wait_timeout(void *stream) {
+    QL_TRY(require_sm100());
+    wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    return launch_check("wait_probe_kernel launch");
+}
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
@@ -571,10 +621,9 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // CTA pairs from 64 tokens up (as the forward); the single-CTA kernel with split-K below that
-    const bool pair = use_pair_fwd(M);
-    const GemmPlan g = plan_gemm(M, K, ceil_div(N, 64));
-    const bool split = !pair && g.splits > 1;
+    // CTA pairs at every M; split-K over n when the output tiles are few
+    const DxPlan g = plan_dx(M, N, K);
+    const bool split = g.splits > 1;
     const WsLayout L = ws_layout(M, K, r, split);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     uint16_t *gs = reinterpret_cast<uint16_t *>(wsb);
@@ -586,51 +635,21 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
         QL_TRY(launch_skinny(dY, 0, B, 1, N, M, r, 1.0f, gacc, r, 1, st));
         QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
     }
+    if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
     const Codebook &cb = codebook_for(w->quant_type);
 
-    if (pair) {
-        const int BN = pair_token_tile(M);
-        CUtensorMap tmY, tmC, tmG;
-        QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
-                            CU_TENSOR_MAP_SWIZZLE_128B));
-        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
-                            CU_TENSOR_MAP_SWIZZLE_64B));
-        if (r > 0)
-            QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
-                                CU_TENSOR_MAP_SWIZZLE_128B));
-        else
-            tmG = tmY;
-        bwdp::Params p;
-        p.scales = w->scales;
-        p.scales2 = w->scales2;
-        p.Alora = A;
-        p.dX = dX;
-        p.M = static_cast<int>(M);
-        p.N = static_cast<int>(N);
-        p.K = static_cast<int>(K);
-        p.r = r;
-        p.BN = BN;
-        for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
-        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel, bwdp::smem_bytes(256)));
-        dim3 grid(static_cast<unsigned>(2 * ceil_div(K, 2 * bwdp::BM)), static_cast<unsigned>(ceil_div(M, BN)), 1);
-        bwdp::fused_bwd_pair_kernel<<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
-        return launch_check("fused_bwd_pair_kernel launch");
-    }
-
-    if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
-
+    const int BN = g.BN;
     CUtensorMap tmY, tmC, tmG;
-    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, g.BN, 64,
+    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, 64, 64,
+    QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
                         CU_TENSOR_MAP_SWIZZLE_64B));
     if (r > 0)
-        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, g.BN, 64,
+        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
                             CU_TENSOR_MAP_SWIZZLE_128B));
     else
         tmG = tmY;
-
-    bwd::Params p;
+    bwdp::Params p;
     p.scales = w->scales;
     p.scales2 = w->scales2;
     p.Alora = A;
@@ -640,18 +659,14 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
     p.r = r;
-    p.BN = g.BN;
-    p.nb_per_split = g.stages_per_split;
+    p.BN = BN;
+    p.nb_per_split = g.nb_per_split;
     for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
-
-    const int smem = bwd::smem_bytes(g.BN);
-    QL_TRY(set_smem(bwd::fused_bwd_dx_kernel, bwd::smem_bytes(256)));
-    dim3 grid(static_cast<unsigned>(g.tiles_rows), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
-    bwd::fused_bwd_dx_kernel<<<grid, bwd::kThreads, smem, st>>>(tmY, tmC, tmG, p);
-    QL_TRY(launch_check("fused_bwd_dx_kernel launch"));
-    if (dxacc) {
-        QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
-    }
+    QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel, bwdp::smem_bytes(256)));
+    dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
+    bwdp::fused_bwd_pair_kernel<<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
+    QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
+    if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
     return QLORA_OK;
 }
 

@@ -219,6 +219,21 @@ qlora_status qlora_sync_status(void *stream);
 /* Message describing the last failure on the calling thread ("" if none). */
 const char *qlora_last_error(void);
 
+/* Sets, on the current device, the time after which any pipeline wait of this
+ * library's kernels gives up (the pages have no counterpart: this is the
+ * failure-detection path of the kernels).  ns must lie in [1e6, 6e10]; the
+ * default is 2e9 (two seconds).  The copy is synchronous: call it with no
+ * kernel of this library in flight and outside stream capture.  QLORA_ERR_ARG
+ * for an out-of-range ns. */
+qlora_status qlora_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of that path: enqueues on `stream` one tiny kernel whose single
+ * pipeline wait has nothing to wait for.  It gives up after the current limit,
+ * records a timeout in the device error word and returns, so the next
+ * qlora_sync_status reports QLORA_ERR_TIMEOUT and clears it; the CUDA context
+ * stays usable.  Nothing else is touched. */
+qlora_status qlora_probe_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

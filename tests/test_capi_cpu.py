@@ -60,6 +60,13 @@ def test_workspace_bytes_covers_adapter_buffer(lib):
     assert lib.qlora_workspace_bytes(0, 1, 1, 8) == 0
 
 
+def test_wait_limit_range_is_checked_on_the_host(lib):
+    # out-of-range limits are refused before any device call
+    assert lib.qlora_set_wait_limit_ns(10) == 1
+    assert "outside" in _err(lib)
+    assert lib.qlora_set_wait_limit_ns(10**12) == 1
+
+
 def _w(n_out=256, n_in=512, codes=0x1000, scales=0x2000, scales2=0x3000):
     return _capi.Nf4WeightC(n_out, n_in, codes, scales, scales2)
 

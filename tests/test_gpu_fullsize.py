@@ -1,11 +1,10 @@
 """Full-size layer shapes on the GPU, checked on sampled outputs the oracle computes one by one.
 
 The 7B FFN pair (with 0.1% outliers, 4096 tokens, r=64) and the 70B shapes run in
-the same launch configuration as every other call.
-- The oracle encodes the whole weight where that stays within seconds.
-- For the 70B FFN matrices it encodes only the 256-block groups that cover the
-  sampled rows. A group is a contiguous run of 16384 weights, so encoding those runs
-  on their own reproduces the full encode of them.
+the same launch configuration as every other call.  The oracle encodes each whole
+weight (about a minute for a 70B FFN matrix), then checks sampled Y columns, sampled
+dX columns, and U, G, dA and dB in full; dA and dB come from the oracle's own chain
+(u = X A^T, g = dY B), never from the GPU's saved factors.
 """
 import numpy as np
 import pytest
@@ -28,26 +27,6 @@ def _assert_tol(got, ref, what):
 
 def _np(t):
     return t.detach().cpu().numpy()
-
-
-def _sampled_rows_oracle(W: torch.Tensor, rows, w_gpu: q.NF4Weight):
-    """Oracle dequant of the given W rows by encoding the groups that cover them; also checks
-    the GPU's codes, u8 scales and fp32 steps of those groups bit for bit."""
-    N, K = W.shape
-    flat = W.reshape(-1)
-    codes_gpu, scales_gpu, s2_gpu = _np(w_gpu.codes), _np(w_gpu.scales), _np(w_gpu.scales2)
-    out = np.empty((len(rows), K), np.float32)
-    for i, r in enumerate(rows):
-        lo, hi = r * K, (r + 1) * K
-        g0, g1 = lo // GROUP_W, (hi - 1) // GROUP_W
-        start, stop = g0 * GROUP_W, min((g1 + 1) * GROUP_W, N * K)
-        ref = O.quantize_nf4_dq(flat[start:stop].numpy())
-        assert np.array_equal(codes_gpu[start // 2:stop // 2], ref["codes"]), f"codes of row {r}"
-        assert np.array_equal(scales_gpu[start // 64:stop // 64], ref["scales"]), f"scales of row {r}"
-        assert np.array_equal(s2_gpu[g0:g1 + 1].view(np.uint32), ref["scales2"].view(np.uint32)), f"steps of row {r}"
-        wd = O.dequant(ref["codes"], ref["scales"], ref["scales2"])
-        out[i] = wd[lo - start:hi - start]
-    return out
 
 
 class Layer:
@@ -90,9 +69,10 @@ def _check_full(layer: Layer, seed: int):
     dXref, gref = O.lora_linear_bwd_dx(Wd[:, cols], dY, A.float().numpy()[:, cols], B, c.scaling)
     _assert_tol(_np(layer.dX.float())[:, cols], dXref, f"{c.name} dX[:, sample]")
     _, uref = O.lora_linear_fwd(np.zeros((1, c.K)), X, A, B, c.scaling)
+    _, gfull = O.lora_linear_bwd_dx(np.zeros((c.N, 1)), dY, A.float().numpy()[:, :1], B, c.scaling)
     _assert_tol(_np(layer.U.float()), uref, f"{c.name} U")
-    _assert_tol(_np(layer.G.float()), gref, f"{c.name} G")
-    dAref, dBref = O.lora_grad_ab(X, dY, layer.U.float().cpu(), layer.G.float().cpu(), c.scaling)
+    _assert_tol(_np(layer.G.float()), gfull, f"{c.name} G")
+    dAref, dBref = O.lora_grad_ab(X, dY, uref, gfull, c.scaling)
     _assert_tol(_np(layer.dA), dAref, f"{c.name} dA")
     _assert_tol(_np(layer.dB), dBref, f"{c.name} dB")
 
@@ -109,13 +89,7 @@ def test_70b_attention_full_size_sampled():
 
 
 @pytest.mark.parametrize("idx", [1, 2], ids=["up-28672x8192", "down-8192x28672"])
-def test_70b_ffn_full_size_sampled_rows(idx):
-    """Forward only; the oracle encodes just the groups of 24 sampled rows."""
-    c = syn.l70b_cases()[idx]
-    layer = Layer(c, with_bwd=False)
-    rng = np.random.default_rng(30 + idx)
-    rows = np.sort(np.concatenate([[0, c.N - 1], rng.choice(np.arange(1, c.N - 1), 22, replace=False)]))
-    Wrows = _sampled_rows_oracle(layer.W, rows, layer.w)
-    X, A, B = (t.cpu() for t in (layer.X, layer.A, layer.B))
-    Yref = O.lora_linear_fwd_rows(Wrows, X, A, B[rows], c.scaling, np.arange(len(rows)))
-    _assert_tol(_np(layer.Y.float())[:, rows], Yref, f"{c.name} Y[:, sample]")
+def test_70b_ffn_full_size_sampled(idx):
+    """Forward and backward of the 70B FFN matrices at 4096 tokens, r = 64."""
+    layer = Layer(syn.l70b_cases()[idx])
+    _check_full(layer, 30 + idx)
