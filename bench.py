@@ -1,24 +1,27 @@
 """Benchmark of the frozen-base NF4 + double-quant LoRA linear layer on B200.
 
-One step = forward (Y, U) + input gradient (dX, G) + adapter gradients (dA, dB)
-of the 7B attention projection: W0 4096x4096 NF4 (blocks of 64, 8-bit double
-quant in groups of 256), 2048 bf16 tokens, LoRA r=8, alpha=16.  Metric:
-algorithmic TFLOP/s = (4MNK + 2Mr(K+N) + 4Mr(N+K)) / step time (the frozen
-base gets no weight gradient).
+One step = forward (Y, U) + input gradient (dX, G) + adapter gradients (dA, dB) of
+every matrix of the 70B-shape layer: attention 8192x8192 and FFN 28672x8192 /
+8192x28672, W0 NF4 (blocks of 64, 8-bit double quant in groups of 256), 4096 bf16
+tokens, LoRA r=64, alpha=128 on every projection.  Metric: algorithmic TFLOP/s =
+sum over the matrices of (4MNK + 2Mr(K+N) + 4Mr(N+K)) / step time (the frozen base
+gets no weight gradient).  The 7B attention (2048 tokens, r=8) and 7B FFN pair
+(4096 tokens, r=64, 0.1 % outliers) are measured the same way beside it, with the
+decode sweep, the one-shot quantize, dequant and merge passes.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1 runs under torchrun as independent replicas (weak scaling, no data-path
 collective); time is the max over ranks.  `--impl reference` times the CPU
-oracle (float64 numpy) on the host cores on a bounded token sample.
+oracle (float64 numpy) on the host cores on a bounded sample of the same layer.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -29,11 +32,30 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fused NF4-dequant LoRA linear TFLOP/s (fwd+bwd)"
-
-# dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kernel on this
-# workload, from one ncu capture each (profiles/); set to None when the kernel changes
-KERNEL_TRAFFIC = {"dx": 25_606_400, "fwd": 25_710_592}
 UNIT = "TFLOP/s"
+CSRC = os.path.join(ROOT, "bit_quantized_base_nf4_b200", "csrc")
+
+# dram__bytes_read.sum + dram__bytes_write.sum of each GEMM kernel, summed over its three
+# launches of one step of the 70B layer, from one ncu capture each (profiles/), with a
+# hash of the kernel sources that capture ran; a source change makes the figure stale
+# and the bench then reports null
+KERNEL_TRAFFIC = {}
+
+
+def kernel_src_hash(kind: str) -> str:
+    files = {"dx": ["fused_bwd_pair.cuh", "ptx.cuh"], "fwd": ["fused_fwd_pair.cuh", "ptx.cuh"]}[kind]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_traffic(kind: str):
+    t = KERNEL_TRAFFIC.get(kind)
+    if not t or t.get("src_sha") != kernel_src_hash(kind):
+        return None
+    return t["bytes"]
 
 
 def algo_flops(M, N, K, r):
@@ -141,26 +163,33 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
-def oracle_sample_step(state):
-    """One oracle pass (fwd + dX + dA/dB in float64) over the sampled tokens."""
-    from oracle import nf4_oracle as O
-    Wd, X, A, B, dY, s = state
-    Y, u = O.lora_linear_fwd(Wd, X, A, B, s)
-    dX, g = O.lora_linear_bwd_dx(Wd, dY, A, B, s)
-    dA, dB = O.lora_grad_ab(X, dY, u, g, s)
-    return Y, dX, dA, dB
+ORACLE_TOKENS, ORACLE_ROWS = 256, 1024
 
 
-def oracle_state(case, m_sample):
+def oracle_sample_step(states):
+    """One oracle pass (fwd + dX + dA/dB in float64) over the sampled sub-layers."""
     from oracle import nf4_oracle as O
-    W = case.weight()
-    ref = O.quantize_nf4_dq(W.numpy())
-    Wd = O.dequant(ref["codes"], ref["scales"], ref["scales2"]).reshape(case.N, case.K).astype(np.float64)
-    X = case.x()[:m_sample].float().numpy().astype(np.float64)
-    dY = case.dy()[:m_sample].float().numpy().astype(np.float64)
-    A = case.lora_a().float().numpy().astype(np.float64)
-    B = case.lora_b().float().numpy().astype(np.float64)
-    return Wd, X, A, B, dY, case.scaling
+    for Wd, X, A, B, dY, s in states:
+        Y, u = O.lora_linear_fwd(Wd, X, A, B, s)
+        dX, g = O.lora_linear_bwd_dx(Wd, dY, A, B, s)
+        O.lora_grad_ab(X, dY, u, g, s)
+
+
+def oracle_states(cases, host):
+    """The oracle's inputs for the bounded sample: for each matrix of the layer, its first
+    ORACLE_ROWS output rows (whole double-quant groups of the row-major weight), encoded and
+    dequantized by the oracle, and the first ORACLE_TOKENS tokens."""
+    from oracle import nf4_oracle as O
+    states, flops = [], 0
+    for c in cases:
+        W, X, A, B, dY = host[c.name]
+        rows = min(ORACLE_ROWS, c.N)
+        ref = O.quantize_nf4_dq(W[:rows].numpy())
+        Wd = O.dequant(ref["codes"], ref["scales"], ref["scales2"]).reshape(rows, c.K).astype(np.float64)
+        f64 = lambda t: t.float().numpy().astype(np.float64)
+        states.append((Wd, f64(X[:ORACLE_TOKENS]), f64(A), f64(B[:rows]), f64(dY[:ORACLE_TOKENS, :rows]), c.scaling))
+        flops += algo_flops(ORACLE_TOKENS, rows, c.K, c.r)
+    return states, flops
 
 
 def blas_threads():
@@ -174,50 +203,59 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(case, m_sample=256, budget_s=10.0):
-    st = oracle_state(case, m_sample)
-    oracle_sample_step(st)                       # warm
+def oracle_sample_desc(cases):
+    return (f"first {ORACLE_ROWS} output rows of each of the {len(cases)} matrices x first {ORACLE_TOKENS} of "
+            f"{cases[0].M} tokens, fwd+dX+dA/dB in float64 numpy")
+
+
+def cpu_baseline(cases, host, budget_s=10.0):
+    states, flops_per_pass = oracle_states(cases, host)
+    oracle_sample_step(states)                       # warm
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_sample_step(st)
+        oracle_sample_step(states)
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     el = time.perf_counter() - t0
-    flops = algo_flops(m_sample, case.N, case.K, case.r) * n
-    return {"value": flops / el / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{m_sample} of {case.M} tokens of {case.name}, fwd+dX+dA/dB in float64 numpy, "
-                      f"{n} passes in {el:.1f} s"}
+    return {"value": flops_per_pass * n / el / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{oracle_sample_desc(cases)}; {n} passes in {el:.1f} s"}
 
 
-def run_reference(args, case):
+def host_tensors(cases):
+    """The seeded synthetic inputs of each matrix, drawn on the host (the tests' bytes)."""
+    return {c.name: (c.weight(), c.x(), c.lora_a(), c.lora_b(), c.dy()) for c in cases}
+
+
+def run_reference(args, cases):
     rank, local, ws = dist_setup("gloo")
     if rank != 0:
         return
-    m_sample = 256
-    st = oracle_state(case, m_sample)
+    host = host_tensors(cases)
+    states, flops_per_pass = oracle_states(cases, host)
     for _ in range(args.warmup):
-        oracle_sample_step(st)
+        oracle_sample_step(states)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_sample_step(st)
+        oracle_sample_step(states)
     el = time.perf_counter() - t0
-    flops = algo_flops(m_sample, case.N, case.K, case.r) * args.steps
-    value = flops / el / 1e12
+    value = flops_per_pass * args.steps / el / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_dict(case, args.gpus),
+            "data": "synthetic", "config": config_dict(cases, args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{m_sample} of {case.M} tokens per step"},
+                             "sample": oracle_sample_desc(cases) + " per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_dict(case, n):
-    return {"workload": f"{case.name}: W0 {case.N}x{case.K} NF4 block 64 + DQ 256, X {case.M}x{case.K} bf16, "
-                        f"LoRA r={case.r} alpha={int(case.alpha)}, fwd + dX + dA/dB",
-            "M": case.M, "N": case.N, "K": case.K, "r": case.r, "alpha": case.alpha,
+def config_dict(cases, n):
+    mats = ", ".join(f"{c.N}x{c.K}" for c in cases)
+    c0 = cases[0]
+    return {"workload": f"70B-shape layer: W0 {{{mats}}} NF4 block 64 + DQ 256, X {c0.M} tokens bf16, "
+                        f"LoRA r={c0.r} alpha={int(c0.alpha)} on every matrix, fwd + dX + dA/dB per matrix",
+            "M": c0.M, "matrices": [[c.N, c.K] for c in cases], "r": c0.r, "alpha": c0.alpha,
             "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{n}"}
 
 
@@ -329,6 +367,35 @@ def quantize_pass(dev, steps, warmup):
             "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
 
 
+def dequant_pass(dev, steps, warmup):
+    """One-shot dequant (the "dequantize the whole matrix" route) of the 70B FFN up
+    projection, 28672 x 8192, to bf16; GB/s = (packed bytes + 2 bytes per weight) / time."""
+    import torch
+    import bit_quantized_base_nf4_b200 as q
+    N, K = 28672, 8192
+    g = torch.Generator(device=dev)
+    g.manual_seed(5150)
+    W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32) * 0.015
+    w = q.NF4Weight.empty(N, K, device=dev)
+    q.qlora_quantize_nf4_dq(W, w)
+    del W
+    out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    for _ in range(warmup):
+        q.qlora_dequant(w, out)
+    a, b = _ev(), _ev()
+    a.record()
+    for _ in range(steps):
+        q.qlora_dequant(w, out)
+    b.record()
+    torch.cuda.synchronize(dev)
+    q.qlora_sync_status()
+    ms = a.elapsed_time(b) / steps
+    nbytes = q.qlora_packed_bytes(N * K) + 2 * N * K
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "70B FFN up 28672x8192 NF4 + DQ -> bf16", "ms": ms, "bytes": nbytes, "GB/s": gbs,
+            "frac_of_hbm": gbs / peaks()["hbm_gbs"]}
+
+
 # ----------------------------------------------------------------------------- merge pass
 
 def merge_pass(dev, steps, warmup):
@@ -382,144 +449,255 @@ def _side_leg(fn):
 
 # ----------------------------------------------------------------------------- CUDA leg
 
-def run_ours(args, case):
+LAUNCHES_PER_MATRIX = 8   # fwd: rank product, finalize, fused GEMM; dX: the same three; dA and dB products
+
+
+class MatrixRun:
+    """Device buffers of one matrix of a layer and its three library calls."""
+
+    def __init__(self, case, host, dev):
+        import torch
+        import bit_quantized_base_nf4_b200 as q
+        self.q, self.c = q, case
+        W, X, A, B, dY = host[case.name]
+        M, N, K, r = case.M, case.N, case.K, case.r
+        self.w = q.NF4Weight.empty(N, K, device=dev)
+        q.qlora_quantize_nf4_dq(W.to(dev), self.w)
+        self.X, self.A, self.B, self.dY = (t.to(dev) for t in (X, A, B, dY))
+        self.ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+        bf = torch.bfloat16
+        self.Y = torch.empty(M, N, dtype=bf, device=dev)
+        self.U = torch.empty(M, r, dtype=bf, device=dev)
+        self.dX = torch.empty(M, K, dtype=bf, device=dev)
+        self.G = torch.empty(M, r, dtype=bf, device=dev)
+        self.dA = torch.empty(r, K, dtype=torch.float32, device=dev)
+        self.dB = torch.empty(N, r, dtype=torch.float32, device=dev)
+        self.flops = algo_flops(M, N, K, r)
+        self.base_flops = 2 * M * N * K
+
+    def fwd(self, st, r=None):
+        c = self.c
+        if r == 0:
+            self.q.qlora_lora_linear_fwd(self.w, self.X, None, None, 0, 0.0, self.Y, None, self.ws, stream=st)
+        else:
+            self.q.qlora_lora_linear_fwd(self.w, self.X, self.A, self.B, c.r, c.scaling, self.Y, self.U, self.ws,
+                                         stream=st)
+
+    def dx(self, st, r=None):
+        c = self.c
+        if r == 0:
+            self.q.qlora_lora_linear_bwd_dx(self.w, self.dY, None, None, 0, 0.0, self.dX, None, self.ws, stream=st)
+        else:
+            self.q.qlora_lora_linear_bwd_dx(self.w, self.dY, self.A, self.B, c.r, c.scaling, self.dX, self.G,
+                                            self.ws, stream=st)
+
+    def grad(self, st):
+        c = self.c
+        self.q.qlora_lora_grad_AB(self.X, self.dY, self.U, self.G, c.r, c.scaling, self.dA, self.dB, stream=st)
+
+
+def _ev():
+    import torch
+    return torch.cuda.Event(enable_timing=True)
+
+
+def measure_layer(runs, dev, st, steps, warmup, flush, clocks=None, e2e=True, kernels=True):
+    """Times `steps` steps (every matrix: fwd, dX, dA/dB) with L2 flushed between steps, then
+    the same step end to end from pinned host memory, then each fused GEMM kernel alone
+    (r = 0 calls: exactly one launch of the kernel).  Returns a dict of measurements."""
+    import torch
+    q = runs[0].q
+    for _ in range(warmup):
+        for m in runs:
+            m.fwd(st); m.dx(st); m.grad(st)
+    q.qlora_sync_status(st)
+    flops = sum(m.flops for m in runs)
+    evs = [[_ev() for _ in range(1 + 3 * len(runs))] for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize(dev)
+    if clocks is not None:
+        clocks.start()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)                         # evict the previous step's operands from L2 (untimed)
+        e = evs[i]
+        e[0].record(st)
+        for j, m in enumerate(runs):
+            m.fwd(st); e[1 + 3 * j].record(st)
+            m.dx(st); e[2 + 3 * j].record(st)
+            m.grad(st); e[3 + 3 * j].record(st)
+    torch.cuda.synchronize(dev)
+    dist_barrier()
+    clk = clocks.stop() if clocks is not None else None
+    q.qlora_sync_status(st)
+    step_ms = [e[0].elapsed_time(e[-1]) for e in evs]
+    ph = {"fwd": 0.0, "bwd_dx": 0.0, "grad_ab": 0.0}
+    per_matrix = {}
+    for j, m in enumerate(runs):
+        f = statistics.mean(e[3 * j].elapsed_time(e[1 + 3 * j]) for e in evs)
+        d = statistics.mean(e[1 + 3 * j].elapsed_time(e[2 + 3 * j]) for e in evs)
+        g = statistics.mean(e[2 + 3 * j].elapsed_time(e[3 + 3 * j]) for e in evs)
+        ph["fwd"] += f; ph["bwd_dx"] += d; ph["grad_ab"] += g
+        per_matrix[m.c.name] = {"fwd_ms": f, "bwd_dx_ms": d, "grad_ab_ms": g,
+                                "TFLOP/s": m.flops / ((f + d + g) * 1e-3) / 1e12}
+    total_ms = dist_max(sum(step_ms), dev)
+    out = {"ms_per_step": total_ms / steps, "flops_per_step": flops,
+           "TFLOP/s": flops / (total_ms / steps * 1e-3) / 1e12, "phases_ms": ph, "per_matrix": per_matrix,
+           "clocks": clk}
+
+    if e2e:
+        # end to end through the same calls with host buffers: H2D of each matrix's X and dY
+        # from pinned memory, the three calls, D2H of dA and dB
+        hosts = [(m.X.cpu().pin_memory(), m.dY.cpu().pin_memory(),
+                  torch.empty_like(m.dA, device="cpu").pin_memory(),
+                  torch.empty_like(m.dB, device="cpu").pin_memory()) for m in runs]
+        e2e_ev = [(_ev(), _ev()) for _ in range(steps)]
+        for i in range(warmup + steps):
+            if i >= warmup:
+                flush.fill_(i & 0xFF)
+                e2e_ev[i - warmup][0].record(st)
+            for m, (hX, hdY, hdA, hdB) in zip(runs, hosts):
+                m.X.copy_(hX, non_blocking=True)
+                m.dY.copy_(hdY, non_blocking=True)
+                m.fwd(st); m.dx(st); m.grad(st)
+                hdA.copy_(m.dA, non_blocking=True)
+                hdB.copy_(m.dB, non_blocking=True)
+            if i >= warmup:
+                e2e_ev[i - warmup][1].record(st)
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status(st)
+        e2e_ms = dist_max(sum(a.elapsed_time(b) for a, b in e2e_ev), dev) / steps
+        out["e2e"] = {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                      "h2d_bytes_per_step": sum((h[0].numel() + h[1].numel()) * 2 for h in hosts),
+                      "d2h_bytes_per_step": sum((h[2].numel() + h[3].numel()) * 4 for h in hosts),
+                      "ms_per_step": e2e_ms}
+        del hosts
+
+    if kernels:
+        # each fused GEMM kernel alone: an r = 0 call is exactly one launch of it
+        kern = {"dx": [], "fwd": []}
+        for i in range(warmup + steps):
+            for m in runs:
+                for kind, call in (("dx", m.dx), ("fwd", m.fwd)):
+                    flush.fill_(i & 0xFF)
+                    a, b = _ev(), _ev()
+                    a.record(st)
+                    call(st, r=0)
+                    b.record(st)
+                    if i >= warmup:
+                        kern[kind].append((m, a, b))
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status(st)
+        pk = peaks()
+        roof = {}
+        for kind, name in (("dx", "fused_bwd_pair_kernel (dX GEMM)"), ("fwd", "fused_fwd_pair_kernel (forward GEMM)")):
+            ms = {}
+            for m, a, b in kern[kind]:
+                ms.setdefault(m.c.name, []).append(a.elapsed_time(b))
+            launch_ms = sum(statistics.mean(v) for v in ms.values())
+            fl = sum(m.base_flops for m in runs)
+            achieved = fl / (launch_ms * 1e-3) / 1e12
+            roof[kind] = {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": achieved / pk["bf16_tflops"], "traffic": kernel_traffic(kind), "kernel": name,
+                          "unit_of_work": f"its {len(runs)} launch(es) of one step, one per matrix (2MNK each)",
+                          "launch_ms": launch_ms, "flops": fl,
+                          "per_matrix_ms": {k: statistics.mean(v) for k, v in ms.items()},
+                          "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json)",
+                          "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"])
+                          if pk.get("bf16_tflops_sustained") else None}
+        out["roofline"] = roof
+    return out
+
+
+def sustained_layer(runs, dev, st, seconds, gpu_index):
+    """Back-to-back steps (no flush) for about `seconds`, with the SM clock sampled: the
+    layer's throughput under the power cap, beside the burst figure."""
+    import torch
+    q = runs[0].q
+    t_one = None
+    clocks = ClockSampler(gpu_index)
+    torch.cuda.synchronize(dev)
+    a, b = _ev(), _ev()
+    a.record(st)
+    for m in runs:
+        m.fwd(st); m.dx(st); m.grad(st)
+    b.record(st)
+    torch.cuda.synchronize(dev)
+    t_one = a.elapsed_time(b)
+    n = max(10, int(seconds * 1e3 / max(t_one, 1e-3)))
+    clocks.start()
+    a.record(st)
+    for _ in range(n):
+        for m in runs:
+            m.fwd(st); m.dx(st); m.grad(st)
+    b.record(st)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    q.qlora_sync_status(st)
+    ms = a.elapsed_time(b) / n
+    flops = sum(m.flops for m in runs)
+    return {"TFLOP/s": flops / (ms * 1e-3) / 1e12, "ms_per_step": ms, "steps": n, "seconds": ms * n / 1e3,
+            "clocks": clk}
+
+
+def run_ours(args, cases):
     import torch
     rank, local, ws = dist_setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    import bit_quantized_base_nf4_b200 as q
-
-    M, N, K, r, s = case.M, case.N, case.K, case.r, case.scaling
-    w = q.NF4Weight.empty(N, K, device=dev)
-    q.qlora_quantize_nf4_dq(case.weight().to(dev), w)
-    X, A, B, dY = (t.to(dev) for t in (case.x(), case.lora_a(), case.lora_b(), case.dy()))
-    wsb = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    U = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    G = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(r, K, dtype=torch.float32, device=dev)
-    dB = torch.empty(N, r, dtype=torch.float32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    from bit_quantized_base_nf4_b200 import synthetic as syn
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 8   # fwd: rank product, finalize, fused GEMM; dX: same three; dA and dB products
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        q.qlora_lora_linear_fwd(w, X, A, B, r, s, Y, U, wsb, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        q.qlora_lora_linear_bwd_dx(w, dY, A, B, r, s, dX, G, wsb, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        q.qlora_lora_grad_AB(X, dY, U, G, r, s, dA, dB, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    q.qlora_sync_status(stream)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    host = host_tensors(cases)
+    runs = [MatrixRun(c, host, dev) for c in cases]
     clocks = ClockSampler(local)
-    dist_barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)                         # evict the previous step's operands from L2 (untimed)
-        step(evs[i])
-    torch.cuda.synchronize(dev)
-    dist_barrier()
-    clk = clocks.stop()
-    q.qlora_sync_status(stream)
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    dx_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    grad_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms = dist_max(sum(step_ms), dev)
-    ms_per_step = total_ms / args.steps
-    value = ws * algo_flops(M, N, K, r) / (ms_per_step * 1e-3) / 1e12
+    head = measure_layer(runs, dev, stream, args.steps, args.warmup, flush, clocks=clocks)
+    value = ws * head["TFLOP/s"]
+    sustained = _side_leg(lambda: sustained_layer(runs, dev, stream, args.sustained_s, local)) \
+        if args.sustained_s > 0 else None
+    del runs
+    torch.cuda.empty_cache()
 
-    # end to end through the same C ABI with host buffers: H2D of the step's inputs from
-    # pinned memory, the three calls, D2H of the adapter gradients.
-    hX, hdY = X.cpu().pin_memory(), dY.cpu().pin_memory()
-    hdA, hdB = torch.empty_like(dA, device="cpu").pin_memory(), torch.empty_like(dB, device="cpu").pin_memory()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for i in range(args.warmup + args.steps):
-        if i >= args.warmup:
-            flush.fill_(i & 0xFF)
-            e2e_ev[i - args.warmup][0].record(stream)
-        X.copy_(hX, non_blocking=True)
-        dY.copy_(hdY, non_blocking=True)
-        step()
-        hdA.copy_(dA, non_blocking=True)
-        hdB.copy_(dB, non_blocking=True)
-        if i >= args.warmup:
-            e2e_ev[i - args.warmup][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = dist_max(sum(a.elapsed_time(b) for a, b in e2e_ev), dev) / args.steps
-    h2d = (hX.numel() + hdY.numel()) * 2
-    d2h = (hdA.numel() + hdB.numel()) * 4
-
-    # the two GEMM kernels alone: with r = 0 each call is exactly one launch of the fused
-    # kernel (dX: CTA-pair transposed-dequant GEMM; forward: CTA-pair dequant GEMM)
-    kern = {"dx": [], "fwd": []}
-    for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xFF)
-        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        a.record(stream)
-        q.qlora_lora_linear_bwd_dx(w, dY, None, None, 0, 0.0, dX, None, wsb, stream=stream)
-        b.record(stream)
-        flush.fill_((i + 1) & 0xFF)
-        b2 = torch.cuda.Event(enable_timing=True)
-        b2.record(stream)
-        q.qlora_lora_linear_fwd(w, X, None, None, 0, 0.0, Y, None, wsb, stream=stream)
-        c.record(stream)
-        if i >= args.warmup:
-            kern["dx"].append((a, b))
-            kern["fwd"].append((b2, c))
-    torch.cuda.synchronize(dev)
-    q.qlora_sync_status(stream)
-    dx_k_ms = statistics.mean(x.elapsed_time(y) for x, y in kern["dx"])
-    fwd_k_ms = statistics.mean(x.elapsed_time(y) for x, y in kern["fwd"])
-    base_flops = 2 * M * N * K
-
-    pk = peaks()
-
-    def roofline(ms, name, traffic):
-        achieved = base_flops / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / pk["bf16_tflops"], "traffic": traffic, "kernel": name,
-                "launch_ms": ms, "flops_per_launch": base_flops,
-                "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json)",
-                "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"])
-                if pk.get("bf16_tflops_sustained") else None}
-
-    # dram bytes per launch from ncu captures of this workload (see profiles/), None once stale
-    roof = roofline(dx_k_ms, "fused_bwd_pair_kernel (dX, dominant kernel of the step)", KERNEL_TRAFFIC.get("dx"))
-    roof_fwd = roofline(fwd_k_ms, "fused_fwd_pair_kernel (forward base GEMM)", KERNEL_TRAFFIC.get("fwd"))
+    # the other layer configurations, measured the same way (no e2e leg)
+    others = {}
+    if not args.headline_only:
+        for label, cs in (("7b_attention_m2048_r8", [syn.attn7b_case()]), ("7b_ffn_pair_m4096_r64", syn.ffn7b_cases())):
+            def leg(cs=cs):
+                h = host_tensors(cs)
+                rr = [MatrixRun(c, h, dev) for c in cs]
+                res = measure_layer(rr, dev, stream, args.steps, args.warmup, flush, e2e=False)
+                res["workload"] = config_dict(cs, ws)["workload"].replace("70B-shape layer", label)
+                return res
+            others[label] = _side_leg(leg)
+            torch.cuda.empty_cache()
 
     if rank == 0:
+        roof = head["roofline"]
+        dominant = max(("dx", "fwd"), key=lambda k: roof[k]["launch_ms"])
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(case, ws),
-                "roofline": roof, "roofline_fwd": roof_fwd,
-                "phases_ms": {"fwd": statistics.mean(fwd_ms), "bwd_dx": statistics.mean(dx_ms),
-                              "grad_ab": statistics.mean(grad_ms)},
-                "e2e": {"value": ws * algo_flops(M, N, K, r) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
-                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-                "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config_dict(cases, ws),
+                "roofline": dict(roof[dominant], dominant_of_step=True),
+                "roofline_other": roof["fwd" if dominant == "dx" else "dx"],
+                "phases_ms": head["phases_ms"], "per_matrix": head["per_matrix"],
+                "e2e": head["e2e"], "gpu_launches": LAUNCHES_PER_MATRIX * len(cases) * args.steps,
+                "clocks": head["clocks"]}
+        if sustained is not None:
+            line["sustained"] = sustained
+        if others:
+            line["configs"] = others
         if not args.no_decode:
             k = max(5, args.steps // 2)
             line["quantize"] = _side_leg(lambda: quantize_pass(dev, k, args.warmup))
+            line["dequant"] = _side_leg(lambda: dequant_pass(dev, k, args.warmup))
             line["decode"] = _side_leg(lambda: decode_sweep(dev, k, args.warmup, args.decode_layers))
             # the configuration's "~6.5e9 weights" counts a gate projection per layer as well
             line["decode_with_gate"] = _side_leg(lambda: decode_sweep(dev, k, args.warmup, args.decode_layers,
                                                                       with_gate=True, ms=(1,)))
             line["merge"] = _side_leg(lambda: merge_pass(dev, 5, args.warmup))
         if ws == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = _side_leg(lambda: cpu_baseline(case))
+            line["cpu_baseline"] = _side_leg(lambda: cpu_baseline(cases, host))
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
     if dist.is_initialized():
@@ -535,7 +713,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
-                    help="skip the quantize, decode-sweep and merge GB/s measurements")
+                    help="skip the quantize, dequant, decode-sweep and merge GB/s measurements")
+    ap.add_argument("--headline-only", action="store_true", help="skip the 7B layer configurations")
+    ap.add_argument("--sustained-s", type=float, default=3.0,
+                    help="seconds of back-to-back steps for the sustained figure (0 skips it)")
     ap.add_argument("--decode-only", action="store_true", help="run only the decode sweep (prints its JSON)")
     ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS)
     ap.add_argument("--merge-only", action="store_true", help="run only the merge + requantize pass (prints its JSON)")
@@ -543,9 +724,9 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     from bit_quantized_base_nf4_b200 import synthetic as syn
-    case = syn.attn7b_case()
+    cases = syn.l70b_cases()
     if args.impl == "reference":
-        run_reference(args, case)
+        run_reference(args, cases)
     elif args.merge_only:
         import torch
         dev = torch.device("cuda", 0)
@@ -557,7 +738,7 @@ def main():
         torch.cuda.set_device(dev)
         print(json.dumps({"decode": decode_sweep(dev, args.steps, args.warmup, args.decode_layers)}), flush=True)
     else:
-        run_ours(args, case)
+        run_ours(args, cases)
 
 
 if __name__ == "__main__":

@@ -15,7 +15,9 @@ import torch
 
 from . import _capi
 
-__all__ = ["NF4Weight", "QLORA_QT_NF4", "QLORA_QT_FP4", "qlora_packed_bytes", "qlora_nf4_codebook", "qlora_codebook",
+__all__ = ["NF4Weight", "QLORA_QT_NF4", "QLORA_QT_FP4", "QLORA_FMT_BLOCK128", "QLORA_FMT_NO_DQ",
+           "QLORA_FMT_CODES_AFTER_DQ", "qlora_packed_bytes", "qlora_packed_bytes_fmt", "qlora_nf4_codebook",
+           "qlora_codebook",
            "qlora_quantize_nf4_dq", "qlora_dequant",
            "qlora_lora_merge_requant",
            "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
@@ -48,35 +50,51 @@ def _need(t, dtype, shape, name):
 
 
 QLORA_QT_NF4, QLORA_QT_FP4 = _capi.QT_NF4, _capi.QT_FP4
+QLORA_FMT_BLOCK128, QLORA_FMT_NO_DQ, QLORA_FMT_CODES_AFTER_DQ = (_capi.FMT_BLOCK128, _capi.FMT_NO_DQ,
+                                                                 _capi.FMT_CODES_AFTER_DQ)
 
 
 @dataclass
 class NF4Weight:
-    """Packed 4-bit weight: device buffers owned by this object (codes, u8 scales, fp32 group
-    steps) and the quant type whose 16 levels the codes index (NF4 by default, or FP4)."""
+    """Packed 4-bit weight: device buffers owned by this object (codes, first-level scales,
+    second-level steps), the quant type whose 16 levels the codes index (NF4 by default, or
+    FP4) and the storage format of the scales (QLORA_FMT_* flags, 0 = blocks of 64 with
+    double quantization).  Without double quantization `scales` holds float32 absmaxes and
+    `scales2` is an empty tensor."""
     n_out: int
     n_in: int
     codes: torch.Tensor
     scales: torch.Tensor
     scales2: torch.Tensor
     quant_type: int = QLORA_QT_NF4
+    format: int = 0
 
     @classmethod
-    def empty(cls, n_out: int, n_in: int, device="cuda", quant_type: int = QLORA_QT_NF4) -> "NF4Weight":
+    def empty(cls, n_out: int, n_in: int, device="cuda", quant_type: int = QLORA_QT_NF4,
+              format: int = 0) -> "NF4Weight":
         numel = n_out * n_in
-        nb = numel // 64
-        return cls(n_out, n_in,
-                   torch.empty(numel // 2, dtype=torch.uint8, device=device),
-                   torch.empty(nb, dtype=torch.uint8, device=device),
-                   torch.empty((nb + 255) // 256, dtype=torch.float32, device=device), int(quant_type))
+        nb = numel // (128 if format & QLORA_FMT_BLOCK128 else 64)
+        if format & QLORA_FMT_NO_DQ:
+            scales = torch.empty(nb, dtype=torch.float32, device=device)
+            scales2 = torch.empty(0, dtype=torch.float32, device=device)
+        else:
+            scales = torch.empty(nb, dtype=torch.uint8, device=device)
+            scales2 = torch.empty((nb + 255) // 256, dtype=torch.float32, device=device)
+        return cls(n_out, n_in, torch.empty(numel // 2, dtype=torch.uint8, device=device), scales, scales2,
+                   int(quant_type), int(format))
 
     def c_struct(self) -> _capi.Nf4WeightC:
-        return _capi.Nf4WeightC(self.n_out, self.n_in, self.codes.data_ptr(), self.scales.data_ptr(),
-                                self.scales2.data_ptr(), int(self.quant_type))
+        s2 = self.scales2.data_ptr() if self.scales2.numel() else None
+        return _capi.Nf4WeightC(self.n_out, self.n_in, self.codes.data_ptr(), self.scales.data_ptr(), s2,
+                                int(self.quant_type), int(self.format))
 
 
 def qlora_packed_bytes(numel: int) -> int:
     return int(_lib().qlora_packed_bytes(int(numel)))
+
+
+def qlora_packed_bytes_fmt(numel: int, format: int) -> int:
+    return int(_lib().qlora_packed_bytes_fmt(int(numel), int(format)))
 
 
 def qlora_nf4_codebook() -> list[float]:

@@ -19,16 +19,19 @@ _vp, _i64, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctyp
 
 class Nf4WeightC(ctypes.Structure):
     _fields_ = [("n_out", ctypes.c_int64), ("n_in", ctypes.c_int64), ("codes", ctypes.c_void_p),
-                ("scales", ctypes.c_void_p), ("scales2", ctypes.c_void_p), ("quant_type", ctypes.c_int32)]
+                ("scales", ctypes.c_void_p), ("scales2", ctypes.c_void_p), ("quant_type", ctypes.c_int32),
+                ("format", ctypes.c_int32)]
 
 
 QT_NF4, QT_FP4 = 0, 1
+FMT_BLOCK128, FMT_NO_DQ, FMT_CODES_AFTER_DQ = 1, 2, 4
 
 
 _WP = ctypes.POINTER(Nf4WeightC)
 
 SIGNATURES = {
     "qlora_packed_bytes": (_sz, [_i64]),
+    "qlora_packed_bytes_fmt": (_sz, [_i64, ctypes.c_int32]),
     "qlora_nf4_codebook": (_int, [ctypes.POINTER(ctypes.c_float)]),
     "qlora_codebook": (_int, [_int, ctypes.POINTER(ctypes.c_float)]),
     "qlora_quantize_nf4_dq": (_int, [_vp, _WP, _vp]),

@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "scale_src.cuh"
 
 namespace qlora {
 namespace bwdp {
@@ -50,8 +51,7 @@ constexpr int kAStageBytes = 64 * BM * 2;     // 64 n x 128 k bf16
 constexpr int kLutWords = 256 * 32;
 
 struct Params {
-    const uint8_t *scales;
-    const float *scales2;
+    ScaleSrc sc;             // first-level scales of the weight's storage format
     const uint16_t *Alora;   // [r, K] bf16 or nullptr
     uint16_t *dX;            // [M, K] bf16 (one split)
     float *dXacc;            // [M, K] fp32 accumulator, zeroed by the host (several splits), or nullptr
@@ -214,18 +214,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t a_off = h * 8192 + nl * 128;
         bool ok = true;
 
-        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
+        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
+        auto load_scale = [&](int s, float &qv, float &dv) {
             const int n = (nb_begin + s) * 64 + nl;
-            qv = 0;
+            qv = 0.f;
             dv = 0.f;
-            if (kvalid && s < NB && n < p.N) {
-                const int64_t b = int64_t(n) * KB + kblk;
-                qv = __ldg(p.scales + b);
-                dv = __ldg(p.scales2 + (b >> 8));
-            }
+            if (kvalid && s < NB && n < p.N) scale_parts(p.sc, int64_t(n) * KB + kblk, qv, dv);
         };
         // block scales of this group's next three stages
-        uint32_t qa, qb, qc;
+        float qa, qb, qc;
         float da, db, dc;
         load_scale(grp, qa, da);
         load_scale(grp + kGroups, qb, db);
@@ -237,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (s < NB) {
                 const int ci = s >> 2, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
-                const float sv = __fmul_rn(static_cast<float>(qa), da);
+                const float sv = __fmul_rn(qa, da);
                 qa = qb; da = db; qb = qc; db = dc;
                 load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);

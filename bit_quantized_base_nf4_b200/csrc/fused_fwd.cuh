@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "scale_src.cuh"
 
 namespace qlora {
 namespace fwd {
@@ -40,8 +41,7 @@ constexpr int kCodeChunkBytes = BM * 128;     // 128 rows x 128 bytes (256 weigh
 constexpr int kLutWords = 256 * 32;           // byte -> bf16x2, replicated per lane
 
 struct Params {
-    const uint8_t *scales;
-    const float *scales2;
+    ScaleSrc sc;             // first-level scales of the weight's storage format
     const uint16_t *Blora;   // [N, r] bf16 or nullptr
     uint16_t *Y;             // [M, N] bf16 (split == 1)
     float *Yacc;             // [M, N] fp32 accumulator (split > 1), zeroed by the host
@@ -199,17 +199,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cswz = row & 7;
         bool ok = true;
         const int64_t row_block0 = int64_t(n) * KB + kb_begin;
-        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
-            qv = 0;
+        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
+        auto load_scale = [&](int s, float &qv, float &dv) {
+            qv = 0.f;
             dv = 0.f;
-            if (valid && s < nmain) {
-                const int64_t b = row_block0 + s;
-                qv = __ldg(p.scales + b);
-                dv = __ldg(p.scales2 + (b >> 8));
-            }
+            if (valid && s < nmain) scale_parts(p.sc, row_block0 + s, qv, dv);
         };
         // block scales of this group's next three stages (12 stages of lookahead)
-        uint32_t qa, qb, qc;
+        float qa, qb, qc;
         float da, db, dc;
         load_scale(grp, qa, da);
         load_scale(grp + kGroups, qb, db);
@@ -220,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t out[32];
             if (s < nmain) {
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
-                const float sv = __fmul_rn(static_cast<float>(qa), da);
+                const float sv = __fmul_rn(qa, da);
                 qa = qb; da = db; qb = qc; db = dc;
                 load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);

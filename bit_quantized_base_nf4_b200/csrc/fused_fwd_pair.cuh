@@ -30,6 +30,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "scale_src.cuh"
 
 namespace qlora {
 namespace fwdp {
@@ -45,8 +46,7 @@ constexpr int kCodeChunkBytes = BM * 128;     // 128 rows x 128 bytes (256 weigh
 constexpr int kLutWords = 256 * 32;           // byte -> bf16x2, replicated per lane
 
 struct Params {
-    const uint8_t *scales;
-    const float *scales2;
+    ScaleSrc sc;             // first-level scales of the weight's storage format
     const uint16_t *Blora;   // [N, r] bf16 or nullptr
     uint16_t *Y;             // [M, N] bf16
     int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
@@ -203,17 +203,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t cswz = row & 7;
         bool ok = true;
         const int64_t row_block0 = int64_t(n) * KB;
-        auto load_scale = [&](int kb, uint32_t &qv, float &dv) {
-            qv = 0;
+        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
+        auto load_scale = [&](int kb, float &qv, float &dv) {
+            qv = 0.f;
             dv = 0.f;
-            if (valid && kb < KB) {
-                const int64_t b = row_block0 + kb;
-                qv = __ldg(p.scales + b);
-                dv = __ldg(p.scales2 + (b >> 8));
-            }
+            if (valid && kb < KB) scale_parts(p.sc, row_block0 + kb, qv, dv);
         };
         // block scales of this group's current and next stage (two 64-blocks each)
-        uint32_t qa0, qa1, qb0, qb1;
+        float qa0, qa1, qb0, qb1;
         float da0, da1, db0, db1;
         load_scale(2 * grp, qa0, da0);
         load_scale(2 * grp + 1, qa1, da1);
@@ -235,8 +232,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint4 c3 = lds128(cbase + (((jq + 3u) ^ cswz) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c_empty[sc]);
-                const float sv0 = __fmul_rn(static_cast<float>(qa0), da0);
-                const float sv1 = __fmul_rn(static_cast<float>(qa1), da1);
+                const float sv0 = __fmul_rn(qa0, da0);
+                const float sv1 = __fmul_rn(qa1, da1);
                 qa0 = qb0; da0 = db0; qa1 = qb1; da1 = db1;
                 load_scale(2 * (q + 2 * kGroups), qb0, db0);
                 load_scale(2 * (q + 2 * kGroups) + 1, qb1, db1);

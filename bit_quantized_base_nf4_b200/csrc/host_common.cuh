@@ -241,14 +241,26 @@ static int sm_count() {
     return n;
 }
 
+// The storage format flags of a weight (QLORA_FMT_*).
+static bool fmt_valid(int32_t f) {
+    return (f & ~(QLORA_FMT_BLOCK128 | QLORA_FMT_NO_DQ | QLORA_FMT_CODES_AFTER_DQ)) == 0 &&
+           !((f & QLORA_FMT_NO_DQ) && (f & QLORA_FMT_CODES_AFTER_DQ));
+}
+static int fmt_block(int32_t f) { return (f & QLORA_FMT_BLOCK128) ? 128 : 64; }
+static bool fmt_dq(int32_t f) { return (f & QLORA_FMT_NO_DQ) == 0; }
+
 static qlora_status check_weight(const qlora_nf4_weight *w) {
     if (!w) return fail(QLORA_ERR_ARG, "weight descriptor is NULL");
+    if (!fmt_valid(w->format))
+        return fail(QLORA_ERR_ARG, "format (%d) is not a valid combination of QLORA_FMT_* flags", w->format);
+    const int blk = fmt_block(w->format);
+    const bool dq = fmt_dq(w->format);
     if (w->n_out <= 0 || w->n_in <= 0) return fail(QLORA_ERR_SHAPE, "n_out and n_in must be positive");
-    if (w->n_in % 64) return fail(QLORA_ERR_SHAPE, "n_in (%lld) must be a multiple of 64", (long long)w->n_in);
+    if (w->n_in % blk) return fail(QLORA_ERR_SHAPE, "n_in (%lld) must be a multiple of the block (%d)", (long long)w->n_in, blk);
     if (w->n_out > (int64_t(1) << 31) || w->n_in > (int64_t(1) << 31))
         return fail(QLORA_ERR_SHAPE, "n_out and n_in must be below 2^31");
-    if (!w->codes || !w->scales || !w->scales2) return fail(QLORA_ERR_ARG, "weight buffers must be non-NULL");
-    if (!aligned16(w->codes) || !aligned16(w->scales) || !aligned16(w->scales2))
+    if (!w->codes || !w->scales || (dq && !w->scales2)) return fail(QLORA_ERR_ARG, "weight buffers must be non-NULL");
+    if (!aligned16(w->codes) || !aligned16(w->scales) || (dq && !aligned16(w->scales2)))
         return fail(QLORA_ERR_ALIGN, "weight buffers must be 16-byte aligned");
     if (w->quant_type != QLORA_QT_NF4 && w->quant_type != QLORA_QT_FP4)
         return fail(QLORA_ERR_ARG, "quant_type (%d) must be QLORA_QT_NF4 (0) or QLORA_QT_FP4 (1)", w->quant_type);

@@ -42,8 +42,19 @@ namespace {
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-static_assert(sizeof(qlora_nf4_weight) == 48 && offsetof(qlora_nf4_weight, quant_type) == 40,
+static_assert(sizeof(qlora_nf4_weight) == 48 && offsetof(qlora_nf4_weight, quant_type) == 40 &&
+                  offsetof(qlora_nf4_weight, format) == 44,
               "the weight descriptor layout is part of the ABI");
+
+// Where the kernels find a weight's first-level scales (see scale_src.cuh).
+ScaleSrc scale_src(const qlora_nf4_weight *w) {
+    ScaleSrc sc;
+    sc.scales = w->scales;
+    sc.scales2 = w->scales2;
+    sc.blk_shift = fmt_block(w->format) == 128 ? 1 : 0;
+    sc.dq = fmt_dq(w->format) ? 1 : 0;
+    return sc;
+}
 
 CodebookArg codebook_arg(int32_t quant_type) {
     CodebookArg a;
@@ -186,11 +197,13 @@ DecodePlan plan_decode(int64_t M, int64_t K, int r) {
 }
 // Small-M forward: the weight-streaming warp-MMA kernel, which needs no workspace,
 // for up to 16 tokens, adapter ranks up to 16 and n_in up to 32768 (when its rings fit).
-bool use_decode(int64_t M, int64_t K, int r) {
-    return M <= 16 && r <= dec::kMaxRank && K / 64 <= dec::kMaxKB && plan_decode(M, K, r).fits;
+// (Default storage format only: other formats take the tensor-core path.)
+bool use_decode(int64_t M, int64_t K, int r, int32_t format) {
+    return format == 0 && M <= 16 && r <= dec::kMaxRank && K / 64 <= dec::kMaxKB && plan_decode(M, K, r).fits;
 }
-size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    if (use_decode(M, K, r)) return 0;
+// format < 0: the largest need over every storage format
+size_t fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r, int32_t format) {
+    if (format >= 0 && use_decode(M, K, r, format)) return 0;
     const bool split = !use_pair_fwd(M) && plan_gemm(M, N, K / 64).splits > 1;
     return ws_layout(M, N, r, split).total;
 }
@@ -332,9 +345,14 @@ qlora_status check_ws(void *ws, size_t ws_bytes, size_t need) {
 
 extern "C" {
 
-size_t qlora_packed_bytes(int64_t numel) {
-    if (numel <= 0 || numel % 64) return 0;
-    const int64_t nb = numel / 64;
+size_t qlora_packed_bytes(int64_t numel) { return qlora_packed_bytes_fmt(numel, 0); }
+
+size_t qlora_packed_bytes_fmt(int64_t numel, int32_t format) {
+    if (!fmt_valid(format)) return 0;
+    const int64_t blk = fmt_block(format);
+    if (numel <= 0 || numel % blk) return 0;
+    const int64_t nb = numel / blk;
+    if (!fmt_dq(format)) return size_t(numel / 2) + 4 * size_t(nb);
     return size_t(numel / 2) + size_t(nb) + 4 * size_t(ceil_div(nb, 256));
 }
 
@@ -372,7 +390,7 @@ qlora_status qlora_probe_wait_timeout(void *stream) {
 
 size_t qlora_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (M <= 0 || N <= 0 || K <= 0) return 0;
-    return std::max<size_t>(256, std::max(fwd_ws_bytes(M, N, K, r), bwd_ws_bytes(M, N, K, r)));
+    return std::max<size_t>(256, std::max(fwd_ws_bytes(M, N, K, r, -1), bwd_ws_bytes(M, N, K, r)));
 }
 
 qlora_status qlora_sync_status(void *stream) {
@@ -395,12 +413,26 @@ qlora_status qlora_quantize_nf4_dq(const float *W, const qlora_nf4_weight *w, vo
     if (!aligned16(W)) return fail(QLORA_ERR_ALIGN, "W must be 16-byte aligned");
     QL_TRY(require_sm100());
     const int64_t numel = w->n_out * w->n_in;
-    const int64_t nblocks = numel / 64;
+    const int blk = fmt_block(w->format);
+    const int64_t nblocks = numel / blk;
     const int64_t ngroups = ceil_div(nblocks, 256);
     if (ngroups > INT32_MAX) return fail(QLORA_ERR_SHAPE, "weight too large");
-    nf4_encode_dq_kernel<<<static_cast<unsigned>(ngroups), kEncThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        W, w->codes, w->scales, w->scales2, nblocks, codebook_arg(w->quant_type));
-    return launch_check("nf4_encode_dq_kernel launch");
+    const dim3 grid(static_cast<unsigned>(ngroups));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const CodebookArg cb = codebook_arg(w->quant_type);
+    const bool dq = fmt_dq(w->format), after = (w->format & QLORA_FMT_CODES_AFTER_DQ) != 0;
+#define QL_ENC(B, D, A) nf4_encode_kernel<B, D, A><<<grid, kEncThreads, 0, st>>>(W, w->codes, w->scales, w->scales2, nblocks, cb)
+    if (blk == 64) {
+        if (!dq) QL_ENC(64, false, false);
+        else if (after) QL_ENC(64, true, true);
+        else QL_ENC(64, true, false);
+    } else {
+        if (!dq) QL_ENC(128, false, false);
+        else if (after) QL_ENC(128, true, true);
+        else QL_ENC(128, true, false);
+    }
+#undef QL_ENC
+    return launch_check("nf4_encode_kernel launch");
 }
 
 qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16, void *stream) {
@@ -409,15 +441,15 @@ qlora_status qlora_dequant(const qlora_nf4_weight *w, void *out, int out_is_bf16
     if (!aligned16(out)) return fail(QLORA_ERR_ALIGN, "out must be 16-byte aligned");
     if (out_is_bf16 != 0 && out_is_bf16 != 1) return fail(QLORA_ERR_ARG, "out_is_bf16 must be 0 or 1");
     QL_TRY(require_sm100());
-    const int64_t n8 = w->n_out * w->n_in / 8;
-    const int64_t grid = std::min<int64_t>(ceil_div(n8, 256), int64_t(sm_count()) * 16);
+    const int64_t n16 = w->n_out * w->n_in / 16;
+    const int64_t grid = std::min<int64_t>(ceil_div(n16, 256), int64_t(sm_count()) * 8);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (out_is_bf16)
-        nf4_dequant_kernel<true><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, w->scales, w->scales2, out,
-                                                                               n8, codebook_arg(w->quant_type));
+        nf4_dequant_kernel<true><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, scale_src(w), out, n16,
+                                                                               codebook_arg(w->quant_type));
     else
-        nf4_dequant_kernel<false><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, w->scales, w->scales2, out,
-                                                                                n8, codebook_arg(w->quant_type));
+        nf4_dequant_kernel<false><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->codes, scale_src(w), out, n16,
+                                                                                codebook_arg(w->quant_type));
     return launch_check("nf4_dequant_kernel launch");
 }
 
@@ -436,7 +468,7 @@ qlora_status qlora_lora_merge_requant(const qlora_nf4_weight *w_in, const qlora_
     const int64_t gy = std::min<int64_t>(w_in->n_out, std::max<int64_t>(1, int64_t(sm_count()) * 16 / gx));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     nf4_lora_merge_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
-        w_in->codes, w_in->scales, w_in->scales2, r > 0 ? reinterpret_cast<const uint16_t *>(A) : nullptr,
+        w_in->codes, scale_src(w_in), r > 0 ? reinterpret_cast<const uint16_t *>(A) : nullptr,
         r > 0 ? reinterpret_cast<const uint16_t *>(B) : nullptr, r, r > 0 ? scaling : 0.f, w_in->n_out, w_in->n_in,
         W_scratch, codebook_arg(w_in->quant_type));
     QL_TRY(launch_check("nf4_lora_merge_kernel launch"));
@@ -453,12 +485,12 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     if (M <= 0 || M > INT32_MAX) return fail(QLORA_ERR_SHAPE, "M (%lld) must be in [1, 2^31)", (long long)M);
     QL_TRY(check_rank(r, scaling, A, B));
     const int64_t N = w->n_out, K = w->n_in;
-    const size_t need = fwd_ws_bytes(M, N, K, r);
+    const size_t need = fwd_ws_bytes(M, N, K, r, w->format);
     QL_TRY(check_ws(ws, ws_bytes, need));
     QL_TRY(require_sm100());
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    if (use_decode(M, K, r)) {
+    if (use_decode(M, K, r, w->format)) {
         DecodePlan d = plan_decode(M, K, r);
         dec::Params &p = d.p;
         p.codes = w->codes;
@@ -534,8 +566,7 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         else
             tmU = tmX;
         fwdp::Params p;
-        p.scales = w->scales;
-        p.scales2 = w->scales2;
+        p.sc = scale_src(w);
         p.Blora = B;
         p.Y = Y;
         p.M = static_cast<int>(M);
@@ -563,8 +594,7 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
         tmU = tmX;
 
     fwd::Params p;
-    p.scales = w->scales;
-    p.scales2 = w->scales2;
+    p.sc = scale_src(w);
     p.Blora = B;
     p.Y = Y;
     p.Yacc = yacc;
@@ -592,7 +622,7 @@ qlora_status qlora_lora_linear_fwd_static_ws(const qlora_nf4_weight *w, const ql
     QL_TRY(check_weight(w));
     if (M <= 0 || M > INT32_MAX) return fail(QLORA_ERR_SHAPE, "M (%lld) must be in [1, 2^31)", (long long)M);
     QL_TRY(check_rank(r, scaling, A, B));
-    const size_t need = fwd_ws_bytes(M, w->n_out, w->n_in, r);
+    const size_t need = fwd_ws_bytes(M, w->n_out, w->n_in, r, w->format);
     if (need > QLORA_STATIC_SCRATCH_BYTES)
         return fail(QLORA_ERR_WORKSPACE,
                     "M=%lld N=%lld K=%lld r=%d needs %zu bytes of scratch; the static scratch holds %zu "
@@ -650,8 +680,7 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     else
         tmG = tmY;
     bwdp::Params p;
-    p.scales = w->scales;
-    p.scales2 = w->scales2;
+    p.sc = scale_src(w);
     p.Alora = A;
     p.dX = dX;
     p.dXacc = dxacc;

@@ -1,11 +1,12 @@
-// quant_kernels.cuh -- NF4 block encode with double quantization of the scales,
-// and the standalone full-tensor dequant.  Both are HBM-bound and bit-exact.
+// quant_kernels.cuh -- 4-bit block encode with (or without) double quantization of the
+// scales, the standalone full-tensor dequant and the LoRA merge.  All are bit-exact.
 #pragma once
 
 #include <cstdint>
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "scale_src.cuh"
 
 namespace qlora {
 
@@ -14,118 +15,170 @@ struct CodebookArg {
     float thresh[16];
 };
 
-// One CTA per group of 256 blocks (16384 weights); 8 warps, each warp walks 32
-// blocks, 4 at a time.  Per block: absmax by warp shuffles, each lane encodes two
-// neighbouring weights into one byte (element 2j low nibble, 2j+1 high nibble).
-// Then the group max gives d_g and each thread quantizes one block scale.
+// Encode.  One CTA per 256 first-level blocks (one double-quant group): 8 warps; a
+// warp step covers 128 consecutive weights, four per lane from one 128-bit load, so a
+// block of 64 spans 16 lanes and a block of 128 the whole warp.  The block absmax is a
+// shuffle reduction over the block's lanes; each lane then encodes its four weights
+// into two code bytes (element 2j low nibble, 2j+1 high nibble).  Then the group max
+// gives d_g and each thread quantizes one block scale (double quant), or stores the
+// fp32 absmax itself (no double quant).  With kAfterDq the codes are taken in a second
+// pass against the dequantized scale s'_b = fp32(q_b d_g) instead of a_b.
 constexpr int kEncThreads = 256;
 
-__global__ void __launch_bounds__(kEncThreads) nf4_encode_dq_kernel(const float *__restrict__ W,
-                                                                    uint8_t *__restrict__ codes,
-                                                                    uint8_t *__restrict__ scales,
-                                                                    float *__restrict__ scales2,
-                                                                    int64_t nblocks, const CodebookArg cb) {
+__device__ __forceinline__ uint32_t code_of(float n, const float *thr) {
+    // #{k : n >= thr[k]} by binary search over the 15 sorted thresholds (thr[15] = inf)
+    uint32_t c = 0;
+    c += (n >= thr[c + 7]) ? 8u : 0u;
+    c += (n >= thr[c + 3]) ? 4u : 0u;
+    c += (n >= thr[c + 1]) ? 2u : 0u;
+    c += (n >= thr[c]) ? 1u : 0u;
+    return c;
+}
+
+__device__ __forceinline__ uint16_t encode4(float4 v, float scale, const float *thr) {
+    float n0 = 0.f, n1 = 0.f, n2 = 0.f, n3 = 0.f;
+    if (scale > 0.f) {
+        n0 = __fdiv_rn(v.x, scale);
+        n1 = __fdiv_rn(v.y, scale);
+        n2 = __fdiv_rn(v.z, scale);
+        n3 = __fdiv_rn(v.w, scale);
+    }
+    const uint32_t c = code_of(n0, thr) | (code_of(n1, thr) << 4) | (code_of(n2, thr) << 8) | (code_of(n3, thr) << 12);
+    return static_cast<uint16_t>(c);
+}
+
+template <int kBlock, bool kDq, bool kAfterDq>
+__global__ void __launch_bounds__(kEncThreads) nf4_encode_kernel(const float *__restrict__ W,
+                                                                 uint8_t *__restrict__ codes,
+                                                                 uint8_t *__restrict__ scales,
+                                                                 float *__restrict__ scales2, int64_t nblocks,
+                                                                 const CodebookArg cb) {
+    static_assert(kBlock == 64 || kBlock == 128, "blocks of 64 or 128 weights");
+    static_assert(kDq || !kAfterDq, "codes against the dequantized scale need double quantization");
+    constexpr int kLanesPerBlock = kBlock / 4;
+    constexpr int kBlocksPerStep = 128 / kBlock;
+    constexpr int U = 4;                           // warp steps in flight
     __shared__ float s_thr[16];
     __shared__ float s_absmax[256];
+    __shared__ float s_scale[kAfterDq ? 256 : 1];
     __shared__ float s_wmax[8];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < 16) s_thr[tid] = cb.thresh[tid];
     const int64_t g = blockIdx.x;
     const int64_t b0 = g * 256;
     const int nb = static_cast<int>(nblocks - b0 < 256 ? nblocks - b0 : 256);
+    const int nsteps = (nb * kBlock + 127) / 128;
+    const float *Wg = W + b0 * kBlock;
+    uint16_t *Cg = reinterpret_cast<uint16_t *>(codes + b0 * (kBlock / 2));
+    const int sub = lane / kLanesPerBlock;         // which block of the step this lane's weights are in
     __syncthreads();
 
-    // encode: warp w handles blocks w*32 .. w*32+31 of the group
-    for (int it = 0; it < 32; it += 4) {
-        float2 v[4];
+    for (int t0 = warp; t0 < nsteps; t0 += 8 * U) {
+        float4 v[U];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int lb = warp * 32 + it + u;
-            v[u] = make_float2(0.f, 0.f);
-            if (lb < nb) v[u] = __ldcs(reinterpret_cast<const float2 *>(W + (b0 + lb) * 64) + lane);
+        for (int u = 0; u < U; ++u) {
+            const int t = t0 + 8 * u;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < nsteps && t * kBlocksPerStep + sub < nb)
+                v[u] = __ldcs(reinterpret_cast<const float4 *>(Wg + int64_t(t) * 128) + lane);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int lb = warp * 32 + it + u;
-            if (lb >= nb) break;  // warp-uniform
-            float a = fmaxf(fabsf(v[u].x), fabsf(v[u].y));
+        for (int u = 0; u < U; ++u) {
+            const int t = t0 + 8 * u;
+            if (t >= nsteps) break;  // warp-uniform
+            const int blk = t * kBlocksPerStep + sub;
+            float a = fmaxf(fmaxf(fabsf(v[u].x), fabsf(v[u].y)), fmaxf(fabsf(v[u].z), fabsf(v[u].w)));
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            float n0 = 0.f, n1 = 0.f;
-            if (a > 0.f) {
-                n0 = __fdiv_rn(v[u].x, a);
-                n1 = __fdiv_rn(v[u].y, a);
+            for (int o = kLanesPerBlock / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            if (blk < nb) {
+                if (!kAfterDq) Cg[t * 32 + lane] = encode4(v[u], a, s_thr);
+                if (lane % kLanesPerBlock == 0) s_absmax[blk] = a;
             }
-            // code = #{k : n >= thresh[k]} by binary search over the 15 sorted thresholds
-            int c0 = 0, c1 = 0;
-            c0 += (n0 >= s_thr[c0 + 7]) ? 8 : 0;
-            c1 += (n1 >= s_thr[c1 + 7]) ? 8 : 0;
-            c0 += (n0 >= s_thr[c0 + 3]) ? 4 : 0;
-            c1 += (n1 >= s_thr[c1 + 3]) ? 4 : 0;
-            c0 += (n0 >= s_thr[c0 + 1]) ? 2 : 0;
-            c1 += (n1 >= s_thr[c1 + 1]) ? 2 : 0;
-            c0 += (n0 >= s_thr[c0]) ? 1 : 0;
-            c1 += (n1 >= s_thr[c1]) ? 1 : 0;
-            codes[(b0 + lb) * 32 + lane] = static_cast<uint8_t>(c0 | (c1 << 4));
-            if (lane == 0) s_absmax[lb] = a;
         }
     }
     __syncthreads();
 
-    // second level: d_g = fp32(max a_b / 255); q_b = clamp(rint(fp32(a_b / d_g)), 0, 255)
-    float a = (tid < nb) ? s_absmax[tid] : 0.f;
-    float m = a;
+    if (kDq) {
+        // second level: d_g = fp32(max a_b / 255); q_b = clamp(rint(fp32(a_b / d_g)), 0, 255)
+        const float a = (tid < nb) ? s_absmax[tid] : 0.f;
+        float m = a;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_wmax[warp] = m;
-    __syncthreads();
-    float c2 = s_wmax[0];
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s_wmax[warp] = m;
+        __syncthreads();
+        float c2 = s_wmax[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) c2 = fmaxf(c2, s_wmax[i]);
-    const float d = __fdiv_rn(c2, 255.f);
-    if (tid < nb) {
-        uint8_t q = 0;
-        if (d > 0.f) {
-            const float r = rintf(__fdiv_rn(a, d));
-            q = static_cast<uint8_t>(fminf(fmaxf(r, 0.f), 255.f));
+        for (int i = 1; i < 8; ++i) c2 = fmaxf(c2, s_wmax[i]);
+        const float d = __fdiv_rn(c2, 255.f);
+        if (tid < nb) {
+            uint32_t q = 0;
+            if (d > 0.f) {
+                const float r = rintf(__fdiv_rn(a, d));
+                q = static_cast<uint32_t>(fminf(fmaxf(r, 0.f), 255.f));
+            }
+            scales[b0 + tid] = static_cast<uint8_t>(q);
+            if (kAfterDq) s_scale[tid] = __fmul_rn(static_cast<float>(q), d);
         }
-        scales[b0 + tid] = q;
+        if (tid == 0) scales2[g] = d;
+    } else {
+        if (tid < nb) reinterpret_cast<float *>(scales)[b0 + tid] = s_absmax[tid];
     }
-    if (tid == 0) scales2[g] = d;
+
+    if (kAfterDq) {
+        __syncthreads();
+        // codes against s'_b: the group's weights again (mostly from L2)
+        for (int t0 = warp; t0 < nsteps; t0 += 8 * U) {
+            float4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int t = t0 + 8 * u;
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (t < nsteps && t * kBlocksPerStep + sub < nb)
+                    v[u] = __ldcs(reinterpret_cast<const float4 *>(Wg + int64_t(t) * 128) + lane);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int t = t0 + 8 * u;
+                if (t >= nsteps) break;
+                const int blk = t * kBlocksPerStep + sub;
+                if (blk < nb) Cg[t * 32 + lane] = encode4(v[u], s_scale[blk], s_thr);
+            }
+        }
+    }
 }
 
-// Full dequant: thread handles 8 weights (4 code bytes).  out_bf16 selects the
-// output type: fp32 w' = fp32(c[code] * fp32(q * d)), or bf16 = RNE(w').
+// Full dequant: a thread handles 16 weights (8 code bytes, one 64-weight run has four
+// threads).  kBf16 selects the output type: fp32 w' = fp32(c[code] * s_b), or
+// bf16 = RNE(w').
 template <bool kBf16>
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes,
-                                                          const uint8_t *__restrict__ scales,
-                                                          const float *__restrict__ scales2,
-                                                          void *__restrict__ out, int64_t n8, const CodebookArg cb) {
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restrict__ codes, const ScaleSrc sc,
+                                                          void *__restrict__ out, int64_t n16, const CodebookArg cb) {
     __shared__ float s_lv[16];
     if (threadIdx.x < 16) s_lv[threadIdx.x] = cb.level[threadIdx.x];
     __syncthreads();
-    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
-        const uint32_t cw = __ldg(reinterpret_cast<const uint32_t *>(codes) + i);
-        const int64_t blk = i >> 3;  // 8 weights per thread, 64 per block
-        const float s = __fmul_rn(static_cast<float>(__ldg(scales + blk)), __ldg(scales2 + (blk >> 8)));
-        float w[8];
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n16; i += int64_t(gridDim.x) * blockDim.x) {
+        const uint2 cw = __ldcs(reinterpret_cast<const uint2 *>(codes) + i);
+        const float s = block_scale(sc, i >> 2);
+        float w[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(s_lv[(cw >> (4 * j)) & 15u], s);
+        for (int j = 0; j < 8; ++j) {
+            w[j] = __fmul_rn(s_lv[(cw.x >> (4 * j)) & 15u], s);
+            w[8 + j] = __fmul_rn(s_lv[(cw.y >> (4 * j)) & 15u], s);
+        }
         if (kBf16) {
-            uint4 o;
-            __nv_bfloat162 p0 = __floats2bfloat162_rn(w[0], w[1]);
-            __nv_bfloat162 p1 = __floats2bfloat162_rn(w[2], w[3]);
-            __nv_bfloat162 p2 = __floats2bfloat162_rn(w[4], w[5]);
-            __nv_bfloat162 p3 = __floats2bfloat162_rn(w[6], w[7]);
-            o.x = *reinterpret_cast<uint32_t *>(&p0);
-            o.y = *reinterpret_cast<uint32_t *>(&p1);
-            o.z = *reinterpret_cast<uint32_t *>(&p2);
-            o.w = *reinterpret_cast<uint32_t *>(&p3);
-            __stcs(reinterpret_cast<uint4 *>(out) + i, o);
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                __nv_bfloat162 p = __floats2bfloat162_rn(w[2 * j], w[2 * j + 1]);
+                o[j] = *reinterpret_cast<uint32_t *>(&p);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(out) + 2 * i;
+            __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
         } else {
-            float4 *o = reinterpret_cast<float4 *>(out) + 2 * i;
-            __stcs(o, make_float4(w[0], w[1], w[2], w[3]));
-            __stcs(o + 1, make_float4(w[4], w[5], w[6], w[7]));
+            float4 *dst = reinterpret_cast<float4 *>(out) + 4 * i;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) __stcs(dst + j, make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
         }
     }
 }
@@ -141,9 +194,7 @@ __device__ __forceinline__ float merge_one(float level, float s, double sd, doub
     const double t = __dadd_rn(static_cast<double>(wb), __dmul_rn(sd, acc));
     return __bfloat162float(__float2bfloat16_rn(__double2float_rn(t)));
 }
-__global__ void __launch_bounds__(256) nf4_lora_merge_kernel(const uint8_t *__restrict__ codes,
-                                                             const uint8_t *__restrict__ scales,
-                                                             const float *__restrict__ scales2,
+__global__ void __launch_bounds__(256) nf4_lora_merge_kernel(const uint8_t *__restrict__ codes, const ScaleSrc sc,
                                                              const uint16_t *__restrict__ A,
                                                              const uint16_t *__restrict__ B, int r, float scaling,
                                                              int64_t N, int64_t K, float *__restrict__ out,
@@ -162,8 +213,7 @@ __global__ void __launch_bounds__(256) nf4_lora_merge_kernel(const uint8_t *__re
             const int64_t i = n * K8 + c;   // code word index; 8 weights per word, 64 per block
             const int64_t k0 = 8 * c;
             const uint32_t cw = __ldg(reinterpret_cast<const uint32_t *>(codes) + i);
-            const int64_t blk = i >> 3;
-            const float s = __fmul_rn(static_cast<float>(__ldg(scales + blk)), __ldg(scales2 + (blk >> 8)));
+            const float s = block_scale(sc, i >> 3);
             double acc[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] = 0.0;

@@ -67,21 +67,37 @@ typedef enum {
  * normalised value takes index 7, a tiny positive one index 8. */
 enum { QLORA_QT_NF4 = 0, QLORA_QT_FP4 = 1 };
 
-/* Packed 4-bit + double-quant weight.  All three buffers are device memory
- * owned by the caller.  numel = n_out * n_in must be a multiple of 64 and
- * n_in must be a multiple of 64 (blocks never straddle rows).
- * quant_type selects the 16 levels (QLORA_QT_NF4 or QLORA_QT_FP4); every call
- * encodes, dequantizes and multiplies with the levels of the weight's type.
- * The descriptor is 48 bytes (the int32 quant_type is followed by padding).
+/* Storage format of the first-level scales, as bit flags ("QLoRA double
+ * quantization ..." page, section 3.1: block size 64 or 128; section 3.2: the
+ * double-quantization switch; sections 1.3 and 2.3 give what each costs).
+ * 0 is the QLoRA default: blocks of 64, double quantization on. */
+enum {
+    QLORA_FMT_BLOCK128 = 1,      /* first-level blocks of 128 weights (n_in % 128 == 0) */
+    QLORA_FMT_NO_DQ = 2,         /* scales are the fp32 block absmaxes; scales2 unused   */
+    QLORA_FMT_CODES_AFTER_DQ = 4 /* encode only: codes are taken against the dequantized
+                                    scale fp32(q_b * d_g) instead of a_b (needs DQ);
+                                    a normalised value beyond +-1 takes the end level    */
+};
+
+/* Packed 4-bit weight.  All buffers are device memory owned by the caller.
+ * With B = 64 (or 128 under QLORA_FMT_BLOCK128): numel = n_out * n_in must be a
+ * multiple of B and n_in a multiple of B (blocks never straddle rows).
+ * quant_type selects the 16 levels (QLORA_QT_NF4 or QLORA_QT_FP4); format the
+ * scale storage (QLORA_FMT_* flags, 0 = default).  Every call encodes,
+ * dequantizes and multiplies with the weight's levels and format.  The
+ * descriptor is 48 bytes.
  *   codes   : numel / 2 bytes; weight element 2j (row-major flattening) is
  *             in bits 0-3 of byte j, element 2j+1 in bits 4-7; each code
  *             indexes the 16 levels of the weight's quant type (see
  *             qlora_codebook).
- *   scales  : numel / 64 bytes; block b (elements [64b, 64b+64)) has first
- *             level scale q_b in 0..255.
- *   scales2 : ceil(numel / 16384) floats; group g (blocks [256g, 256g+256))
- *             has second-level step d_g.  The dequantized block scale is
- *             s_b = fp32(q_b * d_g) and the weight is fp32(c[code] * s_b). */
+ *   scales  : double quant: numel / B bytes; block b (elements [Bb, Bb+B)) has
+ *             first-level scale q_b in 0..255.  No double quant: numel / B
+ *             floats, the block absmax a_b itself.
+ *   scales2 : double quant: ceil(numel / (256 B)) floats; group g (blocks
+ *             [256g, 256g+256)) has second-level step d_g.  Unused (may be
+ *             NULL) without double quant.
+ * The dequantized block scale is s_b = fp32(q_b * d_g) (or a_b) and the weight
+ * is fp32(c[code] * s_b). */
 typedef struct {
     int64_t n_out;
     int64_t n_in;
@@ -89,12 +105,19 @@ typedef struct {
     uint8_t *scales;
     float *scales2;
     int32_t quant_type;
+    int32_t format;
 } qlora_nf4_weight;
 
 /* Bytes of the three packed buffers together: numel/2 + numel/64 +
  * 4*ceil(numel/16384) (the closed form of the "QLoRA double quantization"
  * page, section 2.3).  Returns 0 if numel is not a positive multiple of 64. */
 size_t qlora_packed_bytes(int64_t numel);
+
+/* The same for a storage format (QLORA_FMT_* flags): numel/2 + numel/B +
+ * 4*ceil(numel/(256 B)) with double quantization, numel/2 + 4*numel/B without
+ * (B = 64 or 128).  Returns 0 for a numel that is not a positive multiple of B
+ * or an invalid format. */
+size_t qlora_packed_bytes_fmt(int64_t numel, int32_t format);
 
 /* Writes the 16 NF4 levels (ascending float32, out[0] = -1, out[7] = 0,
  * out[15] = +1) to the HOST array out.  The levels are the normal quantiles
@@ -110,11 +133,14 @@ qlora_status qlora_nf4_codebook(float out[16]);
 qlora_status qlora_codebook(int quant_type, float *out);
 
 /* Encode: W [n_out, n_in] fp32 (device) -> w->codes, w->scales, w->scales2.
- * Per block of 64: a_b = max |w|; code = index of the nearest level to
- * fp32(w / a_b), exact ties to the lower index (a_b = 0 gives code 7).
- * Per group of 256 blocks: d_g = fp32(max a_b / 255) and
- * q_b = clamp(round_half_even(fp32(a_b / d_g)), 0, 255) (d_g = 0 gives 0).
- * Sections 1.2-2.3 of the "QLoRA double quantization" page.  Bit-exact. */
+ * Per block of B (64, or 128 under QLORA_FMT_BLOCK128): a_b = max |w|;
+ * code = index of the level nearest to fp32(w / a_b), exact ties to the lower
+ * index (a_b = 0 gives the code of 0).  Per group of 256 blocks:
+ * d_g = fp32(max a_b / 255) and q_b = clamp(round_half_even(fp32(a_b / d_g)),
+ * 0, 255) (d_g = 0 gives 0).  QLORA_FMT_NO_DQ stores a_b instead of q_b and
+ * d_g; QLORA_FMT_CODES_AFTER_DQ normalises by s_b = fp32(q_b * d_g) instead of
+ * a_b (s_b = 0 gives the code of 0).  Sections 1.2-3.2 of the "QLoRA double
+ * quantization" page.  Bit-exact. */
 qlora_status qlora_quantize_nf4_dq(const float *W, const qlora_nf4_weight *w, void *stream);
 
 /* Dequant the whole weight (the "one-shot dequant" route of the GGUF page,

@@ -162,8 +162,12 @@ def nearest_code(nvals: np.ndarray, book: np.ndarray | None = None) -> np.ndarra
 
     Distances are taken in float64 on the float32 inputs; np.argmin returns
     the first minimum, which is the lower index on an exact tie.  Where a table
-    holds the same value twice (the FP4 table's -0 and +0), a value above it takes
-    the higher copy: the sign of a zero follows the sign of the value.
+    holds the same value twice (the FP4 table's -0 and +0), a value strictly above
+    it takes the higher copy.  That follows from the format, not from a tie rule:
+    an E2M1 number has a sign bit, and round-to-nearest keeps the sign of a
+    strictly positive (negative) value that rounds to zero, giving +0 (-0).  A
+    value that is exactly zero carries no sign here and takes the lower index,
+    the rule of every other exact tie.
     """
     if book is None:
         book = nf4_codebook()
@@ -459,6 +463,14 @@ def lora_merge_bf16(codes, q, d, n_out: int, n_in: int, a, b, scaling: float) ->
     rounded to float32 and then to bf16, the precision the merged base is kept in.
     a [r, K] and b [N, r] are the bf16 adapter factors (any r >= 0)."""
     w = dequant(codes, q, d, n_out * n_in).reshape(n_out, n_in)
+    return lora_merge_bf16_deq(w, a, b, scaling)
+
+
+def lora_merge_bf16_deq(w, a, b, scaling: float) -> np.ndarray:
+    """lora_merge_bf16 from an already dequantized float32 base w [N, K] (any storage
+    format of the packed weight: the steps after the dequant are the same)."""
+    w = np.asarray(w, np.float32)
+    n_out, n_in = w.shape
     wb = bf16_round(w).astype(np.float64)
     acc = np.zeros((n_out, n_in), np.float64)
     a64, b64 = _f64(a), _f64(b)

@@ -60,6 +60,33 @@ def test_workspace_bytes_covers_adapter_buffer(lib):
     assert lib.qlora_workspace_bytes(0, 1, 1, 8) == 0
 
 
+@pytest.mark.parametrize("fmt,block,dq", [(0, 64, True), (1, 128, True), (2, 64, False), (3, 128, False),
+                                          (4, 64, True), (5, 128, True)])
+def test_packed_bytes_of_every_format_matches_closed_form(lib, fmt, block, dq):
+    for n in (128, 16384 * 3, 4096 * 4096, 28672 * 8192):
+        assert lib.qlora_packed_bytes_fmt(n, fmt) == O.packed_bytes_variant(n, block=block, dq=dq)
+    assert lib.qlora_packed_bytes_fmt(64 * 3, 1) == 0          # not a multiple of 128
+    assert lib.qlora_packed_bytes_fmt(128, 6) == 0             # no double quant + codes after it
+    assert lib.qlora_packed_bytes_fmt(128, 8) == 0             # unknown flag
+
+
+def test_format_flags_are_validated(lib):
+    X, Y = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
+    ws = ctypes.c_void_p(0x30000)
+    for fmt, n_in, code, msg in ((8, 512, 1, "format"), (6, 512, 1, "format"), (1, 576, 2, "multiple of the block")):
+        w = _w(n_in=n_in)
+        w.format = fmt
+        st = lib.qlora_lora_linear_fwd(ctypes.byref(w), X, 16, None, None, 0, 0.0, Y, None, ws, 1 << 20, None)
+        assert st == code and msg in _err(lib), (fmt, st, _err(lib))
+    # without double quantization the second-level buffer may be NULL
+    w = _w(scales2=0)
+    w.format = 2
+    st = lib.qlora_dequant(ctypes.byref(w), Y, 0, None)
+    assert st not in (1, 2, 3), _err(lib)       # passes validation (fails later only for want of a GPU)
+    w.format = 0
+    assert lib.qlora_dequant(ctypes.byref(w), Y, 0, None) == 1
+
+
 def test_wait_limit_range_is_checked_on_the_host(lib):
     # out-of-range limits are refused before any device call
     assert lib.qlora_set_wait_limit_ns(10) == 1
@@ -80,7 +107,7 @@ def test_validation_rejects_before_launch(lib):
     assert st == 1 and "NULL" in _err(lib)
     w = _w(n_in=100)
     assert lib.qlora_quantize_nf4_dq(ctypes.c_void_p(0x4000), ctypes.byref(w), None) == 2
-    assert "multiple of 64" in _err(lib)
+    assert "multiple of the block (64)" in _err(lib)
     w = _w(codes=0x1001)
     assert lib.qlora_dequant(ctypes.byref(w), ctypes.c_void_p(0x4000), 0, None) == 3
     w = _w()

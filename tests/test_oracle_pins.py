@@ -726,6 +726,26 @@ def test_q8_0_brute_force_python():
             assert int(got["q"][b * 32 + i]) == want
 
 
+def test_q8_0_float32_quotient_decides_like_the_exact_one():
+    # The kernels divide in float32 (IEEE, correctly rounded) before rounding to an
+    # integer; the oracle divides in float64.  Rounding is monotonic and a half-integer
+    # k + 1/2 below 128 is a float32, so RN32(w / d) reaches it only when w / d equals
+    # it: both precisions round every quotient to the same integer.  Checked here on
+    # weights at and one or two float32 steps around every half-integer tie.
+    rng = np.random.default_rng(93)
+    for _ in range(3000):
+        d = float(np.float16(rng.uniform(1e-5, 2e-3)))
+        k = int(rng.integers(-128, 127))
+        w0 = np.float32((k + 0.5) * d)
+        ws = [w0]
+        for _ in range(2):
+            ws = [np.nextafter(ws[0], np.float32(-1))] + ws + [np.nextafter(ws[-1], np.float32(1))]
+        for w in ws:
+            t64 = float(w) / d
+            t32 = float(np.float32(t64))
+            assert np.rint(t64) == np.rint(t32), (w, d)
+
+
 def test_q8_0_round_trip_bound_and_exact_values():
     rng = np.random.default_rng(92)
     w = (rng.standard_normal(32 * 512) * 0.02).astype(np.float32)
