@@ -453,16 +453,23 @@ LAUNCHES_PER_MATRIX = 8   # fwd: rank product, finalize, fused GEMM; dX: the sam
 
 
 class MatrixRun:
-    """Device buffers of one matrix of a layer and its three library calls."""
+    """Device buffers of one matrix of a layer and its three library calls (NF4 base, or
+    the Q8_0 route with q8=True)."""
 
-    def __init__(self, case, host, dev):
+    def __init__(self, case, host, dev, q8=False):
         import torch
         import bit_quantized_base_nf4_b200 as q
-        self.q, self.c = q, case
+        self.q, self.c, self.q8 = q, case, q8
         W, X, A, B, dY = host[case.name]
         M, N, K, r = case.M, case.N, case.K, case.r
-        self.w = q.NF4Weight.empty(N, K, device=dev)
-        q.qlora_quantize_nf4_dq(W.to(dev), self.w)
+        if q8:
+            self.w = q.Q80Weight.empty(N, K, device=dev)
+            q.qlora_quantize_q8_0(W.to(dev), self.w)
+            self._fwd, self._dx = q.qlora_q8_0_lora_linear_fwd, q.qlora_q8_0_lora_linear_bwd_dx
+        else:
+            self.w = q.NF4Weight.empty(N, K, device=dev)
+            q.qlora_quantize_nf4_dq(W.to(dev), self.w)
+            self._fwd, self._dx = q.qlora_lora_linear_fwd, q.qlora_lora_linear_bwd_dx
         self.X, self.A, self.B, self.dY = (t.to(dev) for t in (X, A, B, dY))
         self.ws = torch.empty(q.qlora_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
         bf = torch.bfloat16
@@ -478,18 +485,16 @@ class MatrixRun:
     def fwd(self, st, r=None):
         c = self.c
         if r == 0:
-            self.q.qlora_lora_linear_fwd(self.w, self.X, None, None, 0, 0.0, self.Y, None, self.ws, stream=st)
+            self._fwd(self.w, self.X, None, None, 0, 0.0, self.Y, None, self.ws, stream=st)
         else:
-            self.q.qlora_lora_linear_fwd(self.w, self.X, self.A, self.B, c.r, c.scaling, self.Y, self.U, self.ws,
-                                         stream=st)
+            self._fwd(self.w, self.X, self.A, self.B, c.r, c.scaling, self.Y, self.U, self.ws, stream=st)
 
     def dx(self, st, r=None):
         c = self.c
         if r == 0:
-            self.q.qlora_lora_linear_bwd_dx(self.w, self.dY, None, None, 0, 0.0, self.dX, None, self.ws, stream=st)
+            self._dx(self.w, self.dY, None, None, 0, 0.0, self.dX, None, self.ws, stream=st)
         else:
-            self.q.qlora_lora_linear_bwd_dx(self.w, self.dY, self.A, self.B, c.r, c.scaling, self.dX, self.G,
-                                            self.ws, stream=st)
+            self._dx(self.w, self.dY, self.A, self.B, c.r, c.scaling, self.dX, self.G, self.ws, stream=st)
 
     def grad(self, st):
         c = self.c
@@ -670,6 +675,18 @@ def run_ours(args, cases):
                 return res
             others[label] = _side_leg(leg)
             torch.cuda.empty_cache()
+
+        # the Q8_0 route (int8 codes, fp16 scale per 32 weights) on the 70B attention matrix
+        def q8_leg():
+            cs = cases[:1]
+            h = {c.name: host[c.name] for c in cs}
+            rr = [MatrixRun(c, h, dev, q8=True) for c in cs]
+            res = measure_layer(rr, dev, stream, args.steps, args.warmup, flush, e2e=False)
+            res["workload"] = (f"Q8_0 route: W0 {cs[0].N}x{cs[0].K} int8 + fp16 scale per 32, X {cs[0].M} tokens bf16, "
+                               f"LoRA r={cs[0].r}, fwd + dX + dA/dB")
+            return res
+        others["q8_0_70b_attention_m4096_r64"] = _side_leg(q8_leg)
+        torch.cuda.empty_cache()
 
     if rank == 0:
         roof = head["roofline"]

@@ -22,7 +22,9 @@ __all__ = ["NF4Weight", "QLORA_QT_NF4", "QLORA_QT_FP4", "QLORA_FMT_BLOCK128", "Q
            "qlora_lora_merge_requant",
            "qlora_workspace_bytes", "qlora_lora_linear_fwd", "qlora_lora_linear_fwd_static_ws",
            "qlora_lora_linear_bwd_dx", "qlora_lora_grad_AB",
-           "qlora_sync_status", "qlora_set_wait_limit_ns", "qlora_probe_wait_timeout", "QloraError"]
+           "qlora_sync_status", "qlora_set_wait_limit_ns", "qlora_probe_wait_timeout", "Q80Weight",
+           "qlora_q8_0_packed_bytes", "qlora_quantize_q8_0", "qlora_dequant_q8_0", "qlora_q8_0_lora_linear_fwd",
+           "qlora_q8_0_lora_linear_bwd_dx", "QloraError"]
 
 QloraError = _capi.QloraError
 
@@ -223,3 +225,75 @@ def qlora_set_wait_limit_ns(ns: int) -> None:
 def qlora_probe_wait_timeout(stream=None) -> None:
     """Enqueue the self-test kernel whose wait runs out; the next sync reports QLORA_ERR_TIMEOUT."""
     _capi.check("qlora_probe_wait_timeout", _lib().qlora_probe_wait_timeout(_stream(stream)))
+
+
+# ----------------------------------------------------------------------------- Q8_0 route
+
+@dataclass
+class Q80Weight:
+    """Q8_0 weight: int8 codes [n_out, n_in] and an fp16 scale per 32 weights (device)."""
+    n_out: int
+    n_in: int
+    q: torch.Tensor
+    d: torch.Tensor
+
+    @classmethod
+    def empty(cls, n_out: int, n_in: int, device="cuda") -> "Q80Weight":
+        return cls(n_out, n_in, torch.empty(n_out * n_in, dtype=torch.int8, device=device),
+                   torch.empty(n_out * n_in // 32, dtype=torch.float16, device=device))
+
+    def c_struct(self) -> _capi.Q80WeightC:
+        return _capi.Q80WeightC(self.n_out, self.n_in, self.q.data_ptr(), self.d.data_ptr())
+
+
+def qlora_q8_0_packed_bytes(numel: int) -> int:
+    return int(_lib().qlora_q8_0_packed_bytes(int(numel)))
+
+
+def qlora_quantize_q8_0(W: torch.Tensor, weight: Q80Weight, stream=None) -> None:
+    _need(W, torch.float32, (weight.n_out, weight.n_in), "W")
+    s = weight.c_struct()
+    _capi.check("qlora_quantize_q8_0", _lib().qlora_quantize_q8_0(_ptr(W), ctypes.byref(s), _stream(stream)))
+
+
+def qlora_dequant_q8_0(weight: Q80Weight, out: torch.Tensor, stream=None) -> None:
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out must be float32 or bfloat16")
+    _need(out, out.dtype, (weight.n_out, weight.n_in), "out")
+    s = weight.c_struct()
+    _capi.check("qlora_dequant_q8_0", _lib().qlora_dequant_q8_0(ctypes.byref(s), _ptr(out),
+                                                                int(out.dtype == torch.bfloat16), _stream(stream)))
+
+
+def qlora_q8_0_lora_linear_fwd(weight: Q80Weight, X, A, B, r: int, scaling: float, Y, U_save=None, ws=None,
+                               stream=None) -> None:
+    M = X.shape[0]
+    _need(X, torch.bfloat16, (M, weight.n_in), "X")
+    _need(Y, torch.bfloat16, (M, weight.n_out), "Y")
+    if r:
+        _need(A, torch.bfloat16, (r, weight.n_in), "A")
+        _need(B, torch.bfloat16, (weight.n_out, r), "B")
+    if U_save is not None:
+        _need(U_save, torch.bfloat16, (M, r), "U_save")
+    s = weight.c_struct()
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    _capi.check("qlora_q8_0_lora_linear_fwd", _lib().qlora_q8_0_lora_linear_fwd(
+        ctypes.byref(s), _ptr(X), M, _ptr(A), _ptr(B), int(r), float(scaling), _ptr(Y), _ptr(U_save), _ptr(ws),
+        wsb, _stream(stream)))
+
+
+def qlora_q8_0_lora_linear_bwd_dx(weight: Q80Weight, dY, A, B, r: int, scaling: float, dX, G_save=None, ws=None,
+                                  stream=None) -> None:
+    M = dY.shape[0]
+    _need(dY, torch.bfloat16, (M, weight.n_out), "dY")
+    _need(dX, torch.bfloat16, (M, weight.n_in), "dX")
+    if r:
+        _need(A, torch.bfloat16, (r, weight.n_in), "A")
+        _need(B, torch.bfloat16, (weight.n_out, r), "B")
+    if G_save is not None:
+        _need(G_save, torch.bfloat16, (M, r), "G_save")
+    s = weight.c_struct()
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    _capi.check("qlora_q8_0_lora_linear_bwd_dx", _lib().qlora_q8_0_lora_linear_bwd_dx(
+        ctypes.byref(s), _ptr(dY), M, _ptr(A), _ptr(B), int(r), float(scaling), _ptr(dX), _ptr(G_save), _ptr(ws),
+        wsb, _stream(stream)))

@@ -29,6 +29,13 @@ FMT_BLOCK128, FMT_NO_DQ, FMT_CODES_AFTER_DQ = 1, 2, 4
 
 _WP = ctypes.POINTER(Nf4WeightC)
 
+
+class Q80WeightC(ctypes.Structure):
+    _fields_ = [("n_out", ctypes.c_int64), ("n_in", ctypes.c_int64), ("q", ctypes.c_void_p), ("d", ctypes.c_void_p)]
+
+
+_QP = ctypes.POINTER(Q80WeightC)
+
 SIGNATURES = {
     "qlora_packed_bytes": (_sz, [_i64]),
     "qlora_packed_bytes_fmt": (_sz, [_i64, ctypes.c_int32]),
@@ -45,6 +52,11 @@ SIGNATURES = {
     "qlora_sync_status": (_int, [_vp]),
     "qlora_last_error": (ctypes.c_char_p, []),
     "qlora_set_wait_limit_ns": (_int, [ctypes.c_uint64]),
+    "qlora_q8_0_packed_bytes": (_sz, [_i64]),
+    "qlora_quantize_q8_0": (_int, [_vp, _QP, _vp]),
+    "qlora_dequant_q8_0": (_int, [_QP, _vp, _int, _vp]),
+    "qlora_q8_0_lora_linear_fwd": (_int, [_QP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "qlora_q8_0_lora_linear_bwd_dx": (_int, [_QP, _vp, _i64, _vp, _vp, _int, _f32, _vp, _vp, _vp, _sz, _vp]),
     "qlora_probe_wait_timeout": (_int, [_vp]),
 }
 

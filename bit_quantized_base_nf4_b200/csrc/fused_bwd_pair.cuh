@@ -28,6 +28,10 @@
 // its own 128 x BN accumulator and writes dX, or, when the contraction over n is
 // split across blockIdx.z (few output tiles: small M), adds it into an fp32
 // accumulator that a finalize kernel rounds to bf16.
+//
+// kQ8 selects the Q8_0 route (GGUF page, sections 1.1 and 2.2): one int8 code per
+// weight and an fp16 scale per 32 weights; a code chunk row then holds 128 bytes
+// (128-byte swizzle) and the dequant threads expand int8 x fp16 scale in registers.
 #pragma once
 
 #include <cstdint>
@@ -51,7 +55,8 @@ constexpr int kAStageBytes = 64 * BM * 2;     // 64 n x 128 k bf16
 constexpr int kLutWords = 256 * 32;
 
 struct Params {
-    ScaleSrc sc;             // first-level scales of the weight's storage format
+    ScaleSrc sc;             // first-level scales of the weight's storage format (4-bit codes)
+    const uint16_t *d8;      // Q8_0: fp16 scale of each 32 weights, [N, K/32]
     const uint16_t *Alora;   // [r, K] bf16 or nullptr
     uint16_t *dX;            // [M, K] bf16 (one split)
     float *dXacc;            // [M, K] fp32 accumulator, zeroed by the host (several splits), or nullptr
@@ -60,16 +65,19 @@ struct Params {
     float level[16];
 };
 
-__host__ __device__ constexpr int smem_bytes(int BN) {
-    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes + kLutWords * 4 + 512;
+__host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
+    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes * (q8 ? 2 : 1) +
+           (q8 ? 0 : kLutWords * 4) + 512;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
     return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u;
 }
 
+template <bool kQ8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fused_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmC,
                           const __grid_constant__ CUtensorMap tmG, const Params p) {
+    constexpr int kCB = kCodeChunkBytes * (kQ8 ? 2 : 1);   // 256 code rows of 64 (4-bit) or 128 (8-bit) bytes
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int half_bn = p.BN / 2;
@@ -77,8 +85,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *sY = smem;
     uint8_t *sA = sY + S * ysb;
     uint8_t *sC = sA + S * kAStageBytes;
-    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
+    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCB);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + (kQ8 ? 0 : kLutWords));
     uint64_t *y_full = bars, *free_b = bars + S;
     uint64_t *c_full = bars + 2 * S, *c_empty = c_full + SC;
     uint64_t *a_full = c_empty + SC;
@@ -126,11 +134,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_relinquish_pair();
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
-        const int e = i >> 5;
-        __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
-        sLut[i] = *reinterpret_cast<uint32_t *>(&v);
-    }
+    if (!kQ8)
+        for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
+            const int e = i >> 5;
+            __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
+            sLut[i] = *reinterpret_cast<uint32_t *>(&v);
+        }
     tc_fence_before();
     // both CTAs' barriers are initialised before either signals the other's
     cluster_sync();
@@ -169,9 +178,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int c = 0; c < nchunk; ++c) {
                 const int sc = c % SC;
                 if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&c_full[sc], kCodeChunkBytes);
-                // rows n = 64 nb_begin + 256c .., bytes k0/2 .. k0/2 + 63
-                tma_load_2d(sC + sc * kCodeChunkBytes, &tmC, &c_full[sc], k0 / 2, nb_begin * 64 + c * kChunkRows);
+                mbar_arrive_expect_tx(&c_full[sc], kCB);
+                // rows n = 64 nb_begin + 256c .., bytes k0/2 .. k0/2 + 63 (4-bit) or k0 .. k0 + 127 (8-bit)
+                tma_load_2d(sC + sc * kCB, &tmC, &c_full[sc], kQ8 ? k0 : k0 / 2, nb_begin * 64 + c * kChunkRows);
                 issued = c + 1;
             }
             for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
@@ -219,8 +228,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int n = (nb_begin + s) * 64 + nl;
             qv = 0.f;
             dv = 0.f;
-            if (kvalid && s < NB && n < p.N) scale_parts(p.sc, int64_t(n) * KB + kblk, qv, dv);
+            if (!kQ8 && kvalid && s < NB && n < p.N) scale_parts(p.sc, int64_t(n) * KB + kblk, qv, dv);
         };
+        // Q8_0: the two fp16 scales of this thread's 64 weights of stage s (as one word)
+        auto load_d8 = [&](int s) -> uint32_t {
+            const int n = (nb_begin + s) * 64 + nl;
+            if (!kQ8 || !kvalid || s >= NB || n >= p.N) return 0u;
+            return __ldg(reinterpret_cast<const uint32_t *>(p.d8 + int64_t(n) * (p.K / 32)) + kblk);
+        };
+        uint32_t ua = load_d8(grp), ub = load_d8(grp + kGroups), uc = load_d8(grp + 2 * kGroups);
         // block scales of this group's next three stages
         float qa, qb, qc;
         float da, db, dc;
@@ -231,7 +247,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = grp; s < total && ok; s += kGroups) {
             const int g = grp;
             uint32_t out[32];
-            if (s < NB) {
+            if (kQ8 && s < NB) {
+                const int ci = s >> 2, sc = ci % SC;
+                if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
+                const uint32_t dd = ua;
+                ua = ub; ub = uc;
+                uc = load_d8(s + 3 * kGroups);
+                // 128-byte code rows, 128-byte swizzle: 16-byte chunk j of row q sits at chunk j ^ (q & 7)
+                const uint32_t cbase = smem_u32(sC) + sc * kCB + ((s & 3) * 64 + nl) * 128;
+                uint4 cv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cv[i] = lds128(cbase + (((4u * h + uint32_t(i)) ^ uint32_t(nl & 7)) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+                const float d_lo = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu)));
+                const float d_hi = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16)));
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float d = v < 2 ? d_lo : d_hi;           // 32 weights per scale
+                    q8_word_to_bf16x2(cv[v].x, d, out[8 * v + 0], out[8 * v + 1]);
+                    q8_word_to_bf16x2(cv[v].y, d, out[8 * v + 2], out[8 * v + 3]);
+                    q8_word_to_bf16x2(cv[v].z, d, out[8 * v + 4], out[8 * v + 5]);
+                    q8_word_to_bf16x2(cv[v].w, d, out[8 * v + 6], out[8 * v + 7]);
+                }
+            } else if (s < NB) {
                 const int ci = s >> 2, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
                 const float sv = __fmul_rn(qa, da);

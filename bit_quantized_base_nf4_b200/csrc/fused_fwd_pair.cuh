@@ -24,6 +24,10 @@
 //   MMA (warp 1, even)   eight tcgen05.mma (K = 16), A from TMEM, B from smem
 // Commits are multicast to both CTAs (free, acc_full).  Each CTA
 // finally reads back its own 128 x BN accumulator.
+//
+// kQ8 selects the Q8_0 route (GGUF page, sections 1.1 and 2.2): one int8 code per
+// weight and an fp16 scale per 32 weights; a code chunk then holds one stage (128 K)
+// and the dequant warps expand int8 x fp16 scale to bf16 in registers (no table).
 #pragma once
 
 #include <cstdint>
@@ -46,22 +50,26 @@ constexpr int kCodeChunkBytes = BM * 128;     // 128 rows x 128 bytes (256 weigh
 constexpr int kLutWords = 256 * 32;           // byte -> bf16x2, replicated per lane
 
 struct Params {
-    ScaleSrc sc;             // first-level scales of the weight's storage format
+    ScaleSrc sc;             // first-level scales of the weight's storage format (4-bit codes)
+    const uint16_t *d8;      // Q8_0: fp16 scale of each 32 weights, [N, K/32]
     const uint16_t *Blora;   // [N, r] bf16 or nullptr
     uint16_t *Y;             // [M, N] bf16
     int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
     float level[16];
 };
 
-__host__ __device__ constexpr int smem_bytes(int BN) {
-    return 1024 /*align slack*/ + SX * 2 * (BN / 2) * 128 + SC * kCodeChunkBytes + kLutWords * 4 + 512 /*barriers*/;
+__host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
+    return 1024 /*align slack*/ + SX * 2 * (BN / 2) * 128 + SC * kCodeChunkBytes + (q8 ? 0 : kLutWords * 4) +
+           512 /*barriers*/;
 }
 // A slots at columns [0, 256), accumulator at [256, 256 + BN)
 __host__ __device__ constexpr uint32_t tmem_cols(int) { return 512u; }
 
+template <bool kQ8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fused_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
                           const __grid_constant__ CUtensorMap tmU, const Params p) {
+    constexpr int kStagesPerChunk = kQ8 ? 1 : 2;   // a 128-byte code row holds 256 (4-bit) or 128 (8-bit) K
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int half_bn = p.BN / 2;
@@ -70,7 +78,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *sX = smem;
     uint8_t *sC = sX + SX * slotb;
     uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + kLutWords);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + (kQ8 ? 0 : kLutWords));
     // stage slot g = q % 4: X slot g and TMEM A slot g share one release barrier free[g]
     uint64_t *x_full = bars, *free_b = bars + SX;
     uint64_t *c_full = bars + 2 * SX, *c_empty = c_full + SC;
@@ -88,7 +96,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int KB = p.K / 64;                      // 64-K chunks of the base
     const int QM = (KB + 1) / 2;                  // main stages
     const int Q = QM + (p.r > 0 ? 1 : 0);         // + one adapter stage (r <= 128)
-    const int nchunk = (KB + 3) / 4;              // 256-K code chunks
+    const int nchunk = (KB + 2 * kStagesPerChunk - 1) / (2 * kStagesPerChunk);   // code chunks
 
     if (threadIdx.x < 16) {
         float v = 0.f;  // constant-index reads keep the parameter block out of local memory
@@ -99,8 +107,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < SX; ++i) { mbar_init(&x_full[i], 1); mbar_init(&free_b[i], 1); }
-        // a chunk is read by the two groups of its two stages
-        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 8); }
+        // a chunk is read by the groups of its stages (four warps each)
+        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 4 * kStagesPerChunk); }
         for (int i = 0; i < kGroups; ++i) mbar_init(&a_full[i], 8);
         mbar_init(acc_full, 1);
         *abort_flag = 0;
@@ -111,11 +119,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_relinquish_pair();
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
-        const int e = i >> 5;
-        __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
-        sLut[i] = *reinterpret_cast<uint32_t *>(&v);
-    }
+    if (!kQ8)
+        for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
+            const int e = i >> 5;
+            __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
+            sLut[i] = *reinterpret_cast<uint32_t *>(&v);
+        }
     tc_fence_before();
     // both CTAs' barriers are initialised before either signals the other's
     cluster_sync();
@@ -207,7 +216,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         auto load_scale = [&](int kb, float &qv, float &dv) {
             qv = 0.f;
             dv = 0.f;
-            if (valid && kb < KB) scale_parts(p.sc, row_block0 + kb, qv, dv);
+            if (!kQ8 && valid && kb < KB) scale_parts(p.sc, row_block0 + kb, qv, dv);
         };
         // block scales of this group's current and next stage (two 64-blocks each)
         float qa0, qa1, qb0, qb1;
@@ -221,7 +230,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int g = grp;
             if (!mbar_wait_cluster(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            if (q < QM) {
+            if (kQ8 && q < QM) {
+                // Q8_0: this stage's 128 code bytes of the row and its four fp16 scales
+                const int sc = q % SC;
+                if (!mbar_wait(&c_full[sc], (q / SC) & 1, abort_flag)) { ok = false; break; }
+                const uint32_t cbase = code_row + sc * kCodeChunkBytes;
+                uint4 cv[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cv[i] = lds128(cbase + ((uint32_t(i) ^ cswz) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+                uint32_t dpair[2] = {0u, 0u};
+                if (valid) {
+                    const uint32_t *drow = reinterpret_cast<const uint32_t *>(p.d8 + int64_t(n) * (p.K / 32));
+                    dpair[0] = __ldg(drow + 2 * q);
+                    if (2 * q + 1 < KB) dpair[1] = __ldg(drow + 2 * q + 1);
+                }
+#pragma unroll
+                for (int sub = 0; sub < 2; ++sub) {
+                    if (sub == 1 && 2 * q + 1 >= KB) break;   // odd last 64-K chunk
+                    uint32_t out[32];
+                    const float d_lo = __half2float(__ushort_as_half(static_cast<unsigned short>(dpair[sub] & 0xFFFFu)));
+                    const float d_hi = __half2float(__ushort_as_half(static_cast<unsigned short>(dpair[sub] >> 16)));
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const uint4 c = cv[4 * sub + v];
+                        const float d = v < 2 ? d_lo : d_hi;       // 32 weights per scale
+                        q8_word_to_bf16x2(c.x, d, out[8 * v + 0], out[8 * v + 1]);
+                        q8_word_to_bf16x2(c.y, d, out[8 * v + 2], out[8 * v + 3]);
+                        q8_word_to_bf16x2(c.z, d, out[8 * v + 4], out[8 * v + 5]);
+                        q8_word_to_bf16x2(c.w, d, out[8 * v + 6], out[8 * v + 7]);
+                    }
+                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                }
+            } else if (q < QM) {
                 const int ci = q >> 1, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
                 const uint32_t cbase = code_row + sc * kCodeChunkBytes;

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace qlora {
 
@@ -283,6 +284,23 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
     __nv_bfloat162 y = *reinterpret_cast<__nv_bfloat162 *>(&b);
     __nv_bfloat162 z = __hmul2(x, y);
     return *reinterpret_cast<uint32_t *>(&z);
+}
+
+// Four int8 codes of one word, times the block scale d, as two bf16x2 words (low byte
+// first).  Each code goes to float32 exactly: flipping its sign bit gives q + 128 in
+// 0..255, placed as the low mantissa byte of 2^23 it reads as 2^23 + q + 128, and
+// subtracting 2^23 + 128 leaves q.  q * d is exact in float32 (8-bit times an fp16
+// significand), then rounds once to bf16.
+__device__ __forceinline__ void q8_word_to_bf16x2(uint32_t w, float d, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const float magic = 8388736.f;   // 2^23 + 128
+    const float f0 = __fmul_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - magic, d);
+    const float f1 = __fmul_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - magic, d);
+    const float f2 = __fmul_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - magic, d);
+    const float f3 = __fmul_rn(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - magic, d);
+    __nv_bfloat162 a = __floats2bfloat162_rn(f0, f1), b = __floats2bfloat162_rn(f2, f3);
+    lo = *reinterpret_cast<uint32_t *>(&a);
+    hi = *reinterpret_cast<uint32_t *>(&b);
 }
 
 // ------------------------------------------------------------------ CTA pairs (cluster of 2)

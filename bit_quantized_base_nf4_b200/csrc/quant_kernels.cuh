@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "ptx.cuh"
 #include "scale_src.cuh"
@@ -179,6 +180,69 @@ __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t *__restr
             float4 *dst = reinterpret_cast<float4 *>(out) + 4 * i;
 #pragma unroll
             for (int j = 0; j < 4; ++j) __stcs(dst + j, make_float4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
+        }
+    }
+}
+
+// Q8_0 encode ("Training LoRA directly on GGUF quantized weights" page, section 1.1:
+// 32 weights share one fp16 scale).  A lane takes four weights (one 128-bit load), so a
+// block spans 8 lanes and a warp step covers 128 weights.  d = fp16(a / 127), taken
+// from the float32 quotient (fp32 keeps 24 >= 2 * 11 + 2 bits, so rounding twice gives
+// the fp16 of the exact quotient); q = clamp(rint(fp32(w / d)), -127, 127); d = 0 gives
+// q = 0.
+__global__ void __launch_bounds__(256) q8_0_encode_kernel(const float *__restrict__ W, int8_t *__restrict__ q,
+                                                          uint16_t *__restrict__ d, int64_t numel) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nsteps = (numel + 127) / 128;
+    for (int64_t t = int64_t(blockIdx.x) * 8 + warp; t < nsteps; t += int64_t(gridDim.x) * 8) {
+        const int64_t e0 = t * 128 + lane * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e0 < numel) v = __ldcs(reinterpret_cast<const float4 *>(W + e0));
+        float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const __half dh = __float2half_rn(__fdiv_rn(a, 127.f));
+        const float df = __half2float(dh);
+        auto code = [&](float x) -> uint32_t {
+            if (!(df > 0.f)) return 0u;
+            const float r = fminf(fmaxf(rintf(__fdiv_rn(x, df)), -127.f), 127.f);
+            return static_cast<uint32_t>(static_cast<int32_t>(r)) & 0xFFu;
+        };
+        if (e0 < numel) {
+            reinterpret_cast<uint32_t *>(q)[e0 >> 2] = code(v.x) | (code(v.y) << 8) | (code(v.z) << 16) | (code(v.w) << 24);
+            if ((lane & 7) == 0) d[e0 >> 5] = __half_as_ushort(dh);
+        }
+    }
+}
+
+// Q8_0 dequant: a thread handles 16 weights (one 128-bit load of codes, one fp16
+// scale): w' = q * d, exact in float32, or bf16 = RNE(w').
+template <bool kBf16>
+__global__ void __launch_bounds__(256) q8_0_dequant_kernel(const int8_t *__restrict__ q,
+                                                           const uint16_t *__restrict__ d, void *__restrict__ out,
+                                                           int64_t n16) {
+    for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < n16; i += int64_t(gridDim.x) * blockDim.x) {
+        const uint4 c = __ldcs(reinterpret_cast<const uint4 *>(q) + i);
+        const float s = __half2float(__ushort_as_half(__ldg(d + (i >> 1))));
+        const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+        if (kBf16) {
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) q8_word_to_bf16x2(words[j], s, o[2 * j], o[2 * j + 1]);
+            uint4 *dst = reinterpret_cast<uint4 *>(out) + 2 * i;
+            __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+        } else {
+            float4 *dst = reinterpret_cast<float4 *>(out) + 4 * i;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int32_t w = static_cast<int32_t>(words[j]);
+                const float f0 = __fmul_rn(static_cast<float>(static_cast<int8_t>(w & 0xFF)), s);
+                const float f1 = __fmul_rn(static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFF)), s);
+                const float f2 = __fmul_rn(static_cast<float>(static_cast<int8_t>((w >> 16) & 0xFF)), s);
+                const float f3 = __fmul_rn(static_cast<float>(static_cast<int8_t>((w >> 24) & 0xFF)), s);
+                __stcs(dst + j, make_float4(f0, f1, f2, f3));
+            }
         }
     }
 }

@@ -236,6 +236,50 @@ qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const
                                 const qlora_bf16 *G, int64_t M, int64_t N, int64_t K, int r,
                                 float scaling, float *dA, float *dB, int accumulate, void *stream);
 
+/* ------------------------------------------------------------------ Q8_0 route
+ * The Q8_0 block format ("Training LoRA directly on GGUF quantized weights"
+ * page, section 1.1: 32 weights share one fp16 scale, a little over one byte
+ * per weight; section 2.2: the blocks are dequantized inside the GEMM, or the
+ * whole matrix at once).  Reading (the page gives no formula): symmetric int8
+ * per block as in the "Quantized vs. non-quantized weights" page, section
+ * 2.1: d = fp16(max |w| / 127), q = clamp(round_half_even(w / d), -127, 127),
+ * w' = q * d (exact in fp32); d = 0 gives q = 0.  The page fixes no byte layout:
+ * the codes and the scales are two row-major arrays.  n_in % 64 == 0.
+ *   q : numel int8 codes, [n_out, n_in] row-major (device)
+ *   d : numel / 32 fp16 scales as IEEE binary16 bit patterns; block b covers
+ *       elements [32b, 32b + 32) of the row-major flattening (device) */
+typedef struct {
+    int64_t n_out;
+    int64_t n_in;
+    int8_t *q;
+    uint16_t *d;
+} qlora_q8_0_weight;
+
+/* numel + 2 * numel / 32 bytes (34 bytes per 32 weights); 0 unless numel is a
+ * positive multiple of 32. */
+size_t qlora_q8_0_packed_bytes(int64_t numel);
+
+/* Encode W [n_out, n_in] fp32 (device) into w->q and w->d, as above.  Bit-exact. */
+qlora_status qlora_quantize_q8_0(const float *W, const qlora_q8_0_weight *w, void *stream);
+
+/* One-shot dequant: out [n_out, n_in] receives q * d as float32 (out_is_bf16 =
+ * 0) or rounded to bfloat16 ties-to-even (1).  Bit-exact. */
+qlora_status qlora_dequant_q8_0(const qlora_q8_0_weight *w, void *out, int out_is_bf16, void *stream);
+
+/* qlora_lora_linear_fwd with a Q8_0 base: the int8 codes and fp16 scales are
+ * expanded in the GEMM main loop to the bf16 operand bf16(q * d).  Same
+ * arguments, rules and workspace (qlora_workspace_bytes covers it). */
+qlora_status qlora_q8_0_lora_linear_fwd(const qlora_q8_0_weight *w, const qlora_bf16 *X, int64_t M,
+                                        const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                        qlora_bf16 *Y, qlora_bf16 *U_save, void *ws, size_t ws_bytes, void *stream);
+
+/* qlora_lora_linear_bwd_dx with a Q8_0 base (the transposed dequant in the main
+ * loop); dA and dB come from qlora_lora_grad_AB as for the 4-bit base. */
+qlora_status qlora_q8_0_lora_linear_bwd_dx(const qlora_q8_0_weight *w, const qlora_bf16 *dY, int64_t M,
+                                           const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                           qlora_bf16 *dX, qlora_bf16 *G_save, void *ws, size_t ws_bytes,
+                                           void *stream);
+
 /* Waits for `stream`, then reports and clears a device-side error recorded by
  * any earlier kernel of this library on the current device: a pipeline wait
  * that timed out (QLORA_ERR_TIMEOUT) or a tensor-memory store whose read-back

@@ -70,6 +70,20 @@ def test_packed_bytes_of_every_format_matches_closed_form(lib, fmt, block, dq):
     assert lib.qlora_packed_bytes_fmt(128, 8) == 0             # unknown flag
 
 
+def test_q8_0_sizes_and_validation(lib):
+    for n in (32, 4096 * 4096, 3_800_000_000 // 32 * 32):
+        assert lib.qlora_q8_0_packed_bytes(n) == O.q8_0_packed_bytes(n)
+    assert lib.qlora_q8_0_packed_bytes(48) == 0
+    w = _capi.Q80WeightC(256, 96, 0x1000, 0x2000)          # n_in not a multiple of 64
+    assert lib.qlora_quantize_q8_0(ctypes.c_void_p(0x4000), ctypes.byref(w), None) == 2
+    w = _capi.Q80WeightC(256, 512, 0x1004, 0x2000)
+    assert lib.qlora_dequant_q8_0(ctypes.byref(w), ctypes.c_void_p(0x4000), 0, None) == 3
+    w = _capi.Q80WeightC(256, 512, 0x1000, 0x2000)
+    X, A, B, Y = (ctypes.c_void_p(a) for a in (0x10000, 0x20000, 0x30000, 0x40000))
+    assert lib.qlora_q8_0_lora_linear_fwd(ctypes.byref(w), X, 16, A, B, 12, 2.0, Y, None, None, 0, None) == 2
+    assert lib.qlora_q8_0_lora_linear_bwd_dx(ctypes.byref(w), X, 64, A, B, 8, 2.0, Y, None, None, 0, None) == 4
+
+
 def test_format_flags_are_validated(lib):
     X, Y = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000)
     ws = ctypes.c_void_p(0x30000)
