@@ -722,6 +722,40 @@ def run_ours(args, cases):
         dist.destroy_process_group()
 
 
+NCU_CASES = {
+    # name: (list of (N, K), M, r, call run per matrix and step)
+    "decode_m1": ([(4096, 4096)], 1, 8, "fwd"),
+    "decode_m16": ([(4096, 4096)], 16, 8, "fwd"),
+    "dx_70b_attn": ([(8192, 8192)], 4096, 0, "dx"),
+    "fwd_70b_attn": ([(8192, 8192)], 4096, 0, "fwd"),
+    # the three matrices of the 70B layer, the GEMM kernel alone (r = 0) once each per step
+    "dx_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "dx"),
+    "fwd_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "fwd"),
+}
+
+
+def ncu_case(name, steps, warmup):
+    """A small, fixed launch sequence for profiler captures: per step, one call of one kind
+    (the forward or dX) on each listed matrix, nothing else after the setup."""
+    import torch
+    import bit_quantized_base_nf4_b200 as q
+    from bit_quantized_base_nf4_b200 import synthetic as syn
+    shapes, M, r, kind = NCU_CASES[name]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    runs = []
+    for i, (N, K) in enumerate(shapes):
+        c = syn.LayerCase(f"{name}-{i}", M=M, N=N, K=K, r=r, alpha=2.0 * r, w_std=0.015, seed=7000 + 10 * i)
+        runs.append(MatrixRun(c, host_tensors([c]), dev))
+    st = torch.cuda.current_stream(dev)
+    for _ in range(warmup + steps):
+        for m in runs:
+            (m.fwd if kind == "fwd" else m.dx)(st)
+    torch.cuda.synchronize(dev)
+    q.qlora_sync_status()
+    print(json.dumps({"ncu_case": name, "calls": (warmup + steps) * len(runs)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -737,12 +771,15 @@ def main():
     ap.add_argument("--decode-only", action="store_true", help="run only the decode sweep (prints its JSON)")
     ap.add_argument("--decode-layers", type=int, default=DECODE_LAYERS)
     ap.add_argument("--merge-only", action="store_true", help="run only the merge + requantize pass (prints its JSON)")
+    ap.add_argument("--ncu-case", choices=sorted(NCU_CASES), help="run one small fixed case for profiler captures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     from bit_quantized_base_nf4_b200 import synthetic as syn
     cases = syn.l70b_cases()
-    if args.impl == "reference":
+    if args.ncu_case:
+        ncu_case(args.ncu_case, args.steps, args.warmup)
+    elif args.impl == "reference":
         run_reference(args, cases)
     elif args.merge_only:
         import torch

@@ -66,8 +66,7 @@ struct Params {
 };
 
 __host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
-    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes * (q8 ? 2 : 1) +
-           (q8 ? 0 : kLutWords * 4) + 512;
+    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes * (q8 ? 2 : 1) + 512;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
     return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u;
@@ -85,8 +84,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *sY = smem;
     uint8_t *sA = sY + S * ysb;
     uint8_t *sC = sA + S * kAStageBytes;
-    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCB);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + (kQ8 ? 0 : kLutWords));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sC + SC * kCB);
     uint64_t *y_full = bars, *free_b = bars + S;
     uint64_t *c_full = bars + 2 * S, *c_empty = c_full + SC;
     uint64_t *a_full = c_empty + SC;
@@ -134,12 +132,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_relinquish_pair();
     }
     __syncthreads();
-    if (!kQ8)
-        for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
-            const int e = i >> 5;
-            __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
-            sLut[i] = *reinterpret_cast<uint32_t *>(&v);
-        }
     tc_fence_before();
     // both CTAs' barriers are initialised before either signals the other's
     cluster_sync();
@@ -215,7 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int h = wi >> 1;                      // k half: columns k0 + 64h ..
         const int kblk = k0 / 64 + h;               // 64-block index along the row
         const bool kvalid = kblk < KB;
-        const uint32_t lut = smem_u32(sLut) + lane * 4;
+        const LevelBytes lvb = level_bytes(*reinterpret_cast<const float (*)[16]>(s_level));
         const uint32_t sAu = smem_u32(sA);
         // 64-byte code rows, 64-byte swizzle: 16-byte chunk c of row q sits at chunk c ^ ((q >> 1) & 3);
         // stage rows start at multiples of 64, so the phase depends on nl only
@@ -284,13 +276,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                // levels from the register byte tables (no shared-memory traffic)
 #pragma unroll
                 for (int w8 = 0; w8 < 8; ++w8) {
+                    codes4_to_bf16x2(words[w8], lvb, out[w8 * 4 + 0], out[w8 * 4 + 1]);
+                    codes4_to_bf16x2(words[w8] >> 16, lvb, out[w8 * 4 + 2], out[w8 * 4 + 3]);
 #pragma unroll
-                    for (int by = 0; by < 4; ++by) {
-                        const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
-                        out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
-                    }
+                    for (int by = 0; by < 4; ++by) out[w8 * 4 + by] = bf16x2_mul(out[w8 * 4 + by], s2);
                 }
             } else {
                 // adapter chunk: row j of A [r, K], 64 k starting at k0 + 64h (zero past r / K)

@@ -58,9 +58,8 @@ struct Params {
     float level[16];
 };
 
-__host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
-    return 1024 /*align slack*/ + SX * 2 * (BN / 2) * 128 + SC * kCodeChunkBytes + (q8 ? 0 : kLutWords * 4) +
-           512 /*barriers*/;
+__host__ __device__ constexpr int smem_bytes(int BN, bool = false) {
+    return 1024 /*align slack*/ + SX * 2 * (BN / 2) * 128 + SC * kCodeChunkBytes + 512 /*barriers*/;
 }
 // A slots at columns [0, 256), accumulator at [256, 256 + BN)
 __host__ __device__ constexpr uint32_t tmem_cols(int) { return 512u; }
@@ -77,8 +76,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int slotb = 2 * xsb;                   // one X ring slot (one stage)
     uint8_t *sX = smem;
     uint8_t *sC = sX + SX * slotb;
-    uint32_t *sLut = reinterpret_cast<uint32_t *>(sC + SC * kCodeChunkBytes);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + (kQ8 ? 0 : kLutWords));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sC + SC * kCodeChunkBytes);
     // stage slot g = q % 4: X slot g and TMEM A slot g share one release barrier free[g]
     uint64_t *x_full = bars, *free_b = bars + SX;
     uint64_t *c_full = bars + 2 * SX, *c_empty = c_full + SC;
@@ -119,12 +117,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_relinquish_pair();
     }
     __syncthreads();
-    if (!kQ8)
-        for (int i = threadIdx.x; i < kLutWords; i += blockDim.x) {
-            const int e = i >> 5;
-            __nv_bfloat162 v = __floats2bfloat162_rn(s_level[e & 15], s_level[e >> 4]);
-            sLut[i] = *reinterpret_cast<uint32_t *>(&v);
-        }
     tc_fence_before();
     // both CTAs' barriers are initialised before either signals the other's
     cluster_sync();
@@ -205,7 +197,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int row = quad * 32 + lane;
         const int n = n0 + row;
         const bool valid = n < p.N;
-        const uint32_t lut = smem_u32(sLut) + lane * 4;
+        const LevelBytes lvb = level_bytes(*reinterpret_cast<const float (*)[16]>(s_level));
         const uint32_t lane_addr = uint32_t(quad * 32) << 16;
         // 128-byte code rows, 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r & 7)
         const uint32_t code_row = smem_u32(sC) + row * 128;
@@ -287,13 +279,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint4 ca = sub ? c2 : c0, cb = sub ? c3 : c1;
                     const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
                     uint32_t out[32];
+                    // levels from the register byte tables (no shared-memory traffic)
 #pragma unroll
                     for (int w8 = 0; w8 < 8; ++w8) {
+                        codes4_to_bf16x2(words[w8], lvb, out[w8 * 4 + 0], out[w8 * 4 + 1]);
+                        codes4_to_bf16x2(words[w8] >> 16, lvb, out[w8 * 4 + 2], out[w8 * 4 + 3]);
 #pragma unroll
-                        for (int by = 0; by < 4; ++by) {
-                            const uint32_t e = (words[w8] >> (8 * by)) & 0xFFu;
-                            out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
-                        }
+                        for (int by = 0; by < 4; ++by) out[w8 * 4 + by] = bf16x2_mul(out[w8 * 4 + by], s2);
                     }
                     tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
                 }

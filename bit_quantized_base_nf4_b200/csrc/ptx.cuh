@@ -303,6 +303,40 @@ __device__ __forceinline__ void q8_word_to_bf16x2(uint32_t w, float d, uint32_t 
     hi = *reinterpret_cast<uint32_t *>(&b);
 }
 
+// The 16 bf16 levels of a 4-bit code as byte tables in registers: hi[i] holds the high
+// bytes of levels 4i .. 4i+3, lo[i] their low bytes.
+struct LevelBytes {
+    uint32_t hi[4], lo[4];
+};
+__device__ __forceinline__ LevelBytes level_bytes(const float (&lv)[16]) {
+    LevelBytes t;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h = 0, l = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const uint32_t u = __bfloat16_as_ushort(__float2bfloat16_rn(lv[4 * i + b]));
+            h |= (u >> 8) << (8 * b);
+            l |= (u & 0xFFu) << (8 * b);
+        }
+        t.hi[i] = h;
+        t.lo[i] = l;
+    }
+    return t;
+}
+// Four 4-bit codes (the low 16 bits of `c`, element j in bits 4j .. 4j+3) to two bf16x2
+// words (elements 0, 1 and 2, 3) by byte permutes on the register tables: each of the
+// four codes picks its byte from levels 0..7 and from 8..15 (low three bits), then bit 3
+// chooses between the two, and the high and low bytes are interleaved.
+__device__ __forceinline__ void codes4_to_bf16x2(uint32_t c, const LevelBytes &t, uint32_t &w01, uint32_t &w23) {
+    const uint32_t sel = c & 0x7777u;
+    const uint32_t pick = ((c >> 1) & 0x4444u) | 0x3210u;
+    const uint32_t h = __byte_perm(__byte_perm(t.hi[0], t.hi[1], sel), __byte_perm(t.hi[2], t.hi[3], sel), pick);
+    const uint32_t l = __byte_perm(__byte_perm(t.lo[0], t.lo[1], sel), __byte_perm(t.lo[2], t.lo[3], sel), pick);
+    w01 = __byte_perm(l, h, 0x5140);
+    w23 = __byte_perm(l, h, 0x7362);
+}
+
 // ------------------------------------------------------------------ CTA pairs (cluster of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

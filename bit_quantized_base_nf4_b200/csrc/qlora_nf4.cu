@@ -332,6 +332,120 @@ qlora_status static_scratch(void **out) {
     return QLORA_OK;
 }
 
+// The packed base weight as the CTA-pair GEMM kernels see it: 4-bit codes with the
+// scales of their storage format and the levels of their quant type, or Q8_0 int8
+// codes with an fp16 scale per 32 weights.
+struct BaseW {
+    const uint8_t *codes;     // [N, K/2] (4-bit) or [N, K] (int8) bytes
+    bool q8;
+    ScaleSrc sc;              // 4-bit only
+    const uint16_t *d8;       // Q8_0 only
+    const float *level;       // 4-bit only: the 16 levels
+};
+
+// Forward base GEMM plus the adapter stage on CTA pairs: Y = X W'^T + us B^T, with
+// us = bf16(scaling * U) [M, r] already in the workspace (r > 0).
+qlora_status launch_fwd_pair(const BaseW &bw, const qlora_bf16 *X, int64_t M, int64_t N, int64_t K,
+                             const qlora_bf16 *B, int r, const uint16_t *us, qlora_bf16 *Y, cudaStream_t st) {
+    const int BN = pair_token_tile(M);
+    CUtensorMap tmX, tmC, tmU;
+    QL_TRY(make_tmap_chunks(&tmX, X, M, K, BN / 2, 2));
+    const uint64_t row_bytes = bw.q8 ? uint64_t(K) : uint64_t(K / 2);
+    QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, row_bytes, row_bytes, 128, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+    if (r > 0)
+        QL_TRY(make_tmap_2d(&tmU, us, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+    else
+        tmU = tmX;
+    fwdp::Params p;
+    p.sc = bw.sc;
+    p.d8 = bw.d8;
+    p.Blora = B;
+    p.Y = Y;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.r = r;
+    p.BN = BN;
+    for (int i = 0; i < 16; ++i) p.level[i] = bw.q8 ? 0.f : bw.level[i];
+    dim3 grid(static_cast<unsigned>(2 * ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, BN)), 1);
+    if (bw.q8) {
+        QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel<true>, fwdp::smem_bytes(256, true)));
+        fwdp::fused_fwd_pair_kernel<true><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN, true), st>>>(tmX, tmC, tmU, p);
+    } else {
+        QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel<false>, fwdp::smem_bytes(256)));
+        fwdp::fused_fwd_pair_kernel<false><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN), st>>>(tmX, tmC, tmU, p);
+    }
+    return launch_check("fused_fwd_pair_kernel launch");
+}
+
+// dX = dY W' + gs A on CTA pairs (gs = bf16(scaling * G) [M, r] in the workspace when
+// r > 0), split over n into dxacc (zeroed by the caller) when the plan says so.
+qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *dY, int64_t M, int64_t N, int64_t K,
+                            const qlora_bf16 *A, int r, const uint16_t *gs, qlora_bf16 *dX, float *dxacc,
+                            cudaStream_t st) {
+    const int BN = g.BN;
+    CUtensorMap tmY, tmC, tmG;
+    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
+                        CU_TENSOR_MAP_SWIZZLE_128B));
+    if (bw.q8)
+        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bwdp::kChunkRows, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+    else
+        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
+                            CU_TENSOR_MAP_SWIZZLE_64B));
+    if (r > 0)
+        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
+                            CU_TENSOR_MAP_SWIZZLE_128B));
+    else
+        tmG = tmY;
+    bwdp::Params p;
+    p.sc = bw.sc;
+    p.d8 = bw.d8;
+    p.Alora = A;
+    p.dX = dX;
+    p.dXacc = dxacc;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.r = r;
+    p.BN = BN;
+    p.nb_per_split = g.nb_per_split;
+    for (int i = 0; i < 16; ++i) p.level[i] = bw.q8 ? 0.f : bw.level[i];
+    dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
+    if (bw.q8) {
+        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<true>, bwdp::smem_bytes(256, true)));
+        bwdp::fused_bwd_pair_kernel<true><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN, true), st>>>(tmY, tmC, tmG, p);
+    } else {
+        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<false>, bwdp::smem_bytes(256)));
+        bwdp::fused_bwd_pair_kernel<false><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
+    }
+    QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
+    if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
+    return QLORA_OK;
+}
+
+// The rank-r side product of the forward (U = X A^T: us = bf16(scaling U), U_save = bf16(U))
+// or of dX (G = dY B), into the workspace.
+qlora_status rank_side_product(bool fwd, const qlora_bf16 *act, int64_t M, int64_t width, const qlora_bf16 *factor,
+                               int r, float scaling, uint16_t *scaled, float *acc, qlora_bf16 *save, cudaStream_t st) {
+    QL_TRY(cuda_check(cudaMemsetAsync(acc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
+    if (fwd) QL_TRY(launch_skinny(act, 0, factor, 0, width, M, r, 1.0f, acc, r, 1, st));
+    else QL_TRY(launch_skinny(act, 0, factor, 1, width, M, r, 1.0f, acc, r, 1, st));
+    return launch_finalize(acc, M * r, scaling, save, scaled, st);
+}
+
+BaseW base_of(const qlora_nf4_weight *w, const Codebook &cb) {
+    BaseW b;
+    b.codes = w->codes;
+    b.q8 = false;
+    b.sc = scale_src(w);
+    b.d8 = nullptr;
+    b.level = cb.level;
+    return b;
+}
+
 qlora_status check_ws(void *ws, size_t ws_bytes, size_t need) {
     if (need == 0) return QLORA_OK;
     if (!ws) return fail(QLORA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
@@ -546,40 +660,11 @@ qlora_status qlora_lora_linear_fwd(const qlora_nf4_weight *w, const qlora_bf16 *
     uint16_t *us = reinterpret_cast<uint16_t *>(wsb);
     float *uacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
     float *yacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
-    if (r > 0) {
-        // U = X A^T on tensor cores, then bf16 copies: U (saved) and scaling * U (adapter chunk)
-        QL_TRY(cuda_check(cudaMemsetAsync(uacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
-        QL_TRY(launch_skinny(X, 0, A, 0, K, M, r, 1.0f, uacc, r, 1, st));
-        QL_TRY(launch_finalize(uacc, M * r, scaling, U_save, us, st));
-    }
+    // U = X A^T on tensor cores, then bf16 copies: U (saved) and scaling * U (adapter chunk)
+    if (r > 0) QL_TRY(rank_side_product(true, X, M, K, A, r, scaling, us, uacc, U_save, st));
     const Codebook &cb = codebook_for(w->quant_type);
 
-    if (pair) {
-        const int BN = pair_token_tile(M);
-        CUtensorMap tmX, tmC, tmU;
-        QL_TRY(make_tmap_chunks(&tmX, X, M, K, BN / 2, 2));
-        QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, 128, 128,
-                            CU_TENSOR_MAP_SWIZZLE_128B));
-        if (r > 0)
-            QL_TRY(make_tmap_2d(&tmU, us, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
-                                CU_TENSOR_MAP_SWIZZLE_128B));
-        else
-            tmU = tmX;
-        fwdp::Params p;
-        p.sc = scale_src(w);
-        p.Blora = B;
-        p.Y = Y;
-        p.M = static_cast<int>(M);
-        p.N = static_cast<int>(N);
-        p.K = static_cast<int>(K);
-        p.r = r;
-        p.BN = BN;
-        for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
-        QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel, fwdp::smem_bytes(256)));
-        dim3 grid(static_cast<unsigned>(2 * ceil_div(N, 256)), static_cast<unsigned>(ceil_div(M, BN)), 1);
-        fwdp::fused_fwd_pair_kernel<<<grid, fwdp::kThreads, fwdp::smem_bytes(BN), st>>>(tmX, tmC, tmU, p);
-        return launch_check("fused_fwd_pair_kernel launch");
-    }
+    if (pair) return launch_fwd_pair(base_of(w, cb), X, M, N, K, B, r, us, Y, st);
 
     if (yacc) QL_TRY(cuda_check(cudaMemsetAsync(yacc, 0, size_t(M) * N * 4, st), "zero split accumulator"));
     CUtensorMap tmX, tmC, tmU;
@@ -659,44 +744,115 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     uint16_t *gs = reinterpret_cast<uint16_t *>(wsb);
     float *gacc = reinterpret_cast<float *>(wsb + L.rank_bf16);
     float *dxacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
-    if (r > 0) {
-        // G = dY B on tensor cores (B read MN-major), then bf16 copies G and scaling * G
-        QL_TRY(cuda_check(cudaMemsetAsync(gacc, 0, size_t(M) * r * 4, st), "zero rank accumulator"));
-        QL_TRY(launch_skinny(dY, 0, B, 1, N, M, r, 1.0f, gacc, r, 1, st));
-        QL_TRY(launch_finalize(gacc, M * r, scaling, G_save, gs, st));
-    }
+    // G = dY B on tensor cores (B read MN-major), then bf16 copies G and scaling * G
+    if (r > 0) QL_TRY(rank_side_product(false, dY, M, N, B, r, scaling, gs, gacc, G_save, st));
     if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
-    const Codebook &cb = codebook_for(w->quant_type);
+    return launch_dx_pair(base_of(w, codebook_for(w->quant_type)), g, dY, M, N, K, A, r, gs, dX, dxacc, st);
+}
 
-    const int BN = g.BN;
-    CUtensorMap tmY, tmC, tmG;
-    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B));
-    QL_TRY(make_tmap_2d(&tmC, w->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
-                        CU_TENSOR_MAP_SWIZZLE_64B));
-    if (r > 0)
-        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
-                            CU_TENSOR_MAP_SWIZZLE_128B));
-    else
-        tmG = tmY;
-    bwdp::Params p;
-    p.sc = scale_src(w);
-    p.Alora = A;
-    p.dX = dX;
-    p.dXacc = dxacc;
-    p.M = static_cast<int>(M);
-    p.N = static_cast<int>(N);
-    p.K = static_cast<int>(K);
-    p.r = r;
-    p.BN = BN;
-    p.nb_per_split = g.nb_per_split;
-    for (int i = 0; i < 16; ++i) p.level[i] = cb.level[i];
-    QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel, bwdp::smem_bytes(256)));
-    dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
-    bwdp::fused_bwd_pair_kernel<<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
-    QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
-    if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
+// ------------------------------------------------------------------ Q8_0 route
+
+static qlora_status check_q8(const qlora_q8_0_weight *w) {
+    if (!w) return fail(QLORA_ERR_ARG, "weight descriptor is NULL");
+    if (w->n_out <= 0 || w->n_in <= 0) return fail(QLORA_ERR_SHAPE, "n_out and n_in must be positive");
+    if (w->n_in % 64) return fail(QLORA_ERR_SHAPE, "n_in (%lld) must be a multiple of 64", (long long)w->n_in);
+    if (w->n_out > (int64_t(1) << 31) || w->n_in > (int64_t(1) << 31))
+        return fail(QLORA_ERR_SHAPE, "n_out and n_in must be below 2^31");
+    if (!w->q || !w->d) return fail(QLORA_ERR_ARG, "weight buffers must be non-NULL");
+    if (!aligned16(w->q) || !aligned16(w->d)) return fail(QLORA_ERR_ALIGN, "weight buffers must be 16-byte aligned");
     return QLORA_OK;
+}
+
+static BaseW base_of_q8(const qlora_q8_0_weight *w) {
+    BaseW b;
+    b.codes = reinterpret_cast<const uint8_t *>(w->q);
+    b.q8 = true;
+    b.sc = ScaleSrc{nullptr, nullptr, 0, 1};
+    b.d8 = w->d;
+    b.level = nullptr;
+    return b;
+}
+
+size_t qlora_q8_0_packed_bytes(int64_t numel) {
+    if (numel <= 0 || numel % 32) return 0;
+    return size_t(numel) + 2 * size_t(numel / 32);
+}
+
+qlora_status qlora_quantize_q8_0(const float *W, const qlora_q8_0_weight *w, void *stream) {
+    QL_TRY(check_q8(w));
+    if (!W) return fail(QLORA_ERR_ARG, "W is NULL");
+    if (!aligned16(W)) return fail(QLORA_ERR_ALIGN, "W must be 16-byte aligned");
+    QL_TRY(require_sm100());
+    const int64_t numel = w->n_out * w->n_in;
+    const int64_t grid = std::min<int64_t>(ceil_div(ceil_div(numel, 128), 8), int64_t(sm_count()) * 16);
+    q8_0_encode_kernel<<<static_cast<unsigned>(grid), 256, 0, static_cast<cudaStream_t>(stream)>>>(W, w->q, w->d,
+                                                                                                 numel);
+    return launch_check("q8_0_encode_kernel launch");
+}
+
+qlora_status qlora_dequant_q8_0(const qlora_q8_0_weight *w, void *out, int out_is_bf16, void *stream) {
+    QL_TRY(check_q8(w));
+    if (!out) return fail(QLORA_ERR_ARG, "out is NULL");
+    if (!aligned16(out)) return fail(QLORA_ERR_ALIGN, "out must be 16-byte aligned");
+    if (out_is_bf16 != 0 && out_is_bf16 != 1) return fail(QLORA_ERR_ARG, "out_is_bf16 must be 0 or 1");
+    QL_TRY(require_sm100());
+    const int64_t n16 = w->n_out * w->n_in / 16;
+    const int64_t grid = std::min<int64_t>(ceil_div(n16, 256), int64_t(sm_count()) * 8);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (out_is_bf16) q8_0_dequant_kernel<true><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->q, w->d, out, n16);
+    else q8_0_dequant_kernel<false><<<static_cast<unsigned>(grid), 256, 0, st>>>(w->q, w->d, out, n16);
+    return launch_check("q8_0_dequant_kernel launch");
+}
+
+qlora_status qlora_q8_0_lora_linear_fwd(const qlora_q8_0_weight *w, const qlora_bf16 *X, int64_t M,
+                                        const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                        qlora_bf16 *Y, qlora_bf16 *U_save, void *ws, size_t ws_bytes, void *stream) {
+    QL_TRY(check_q8(w));
+    if (!X || !Y) return fail(QLORA_ERR_ARG, "X and Y must be non-NULL");
+    if (!aligned16(X) || !aligned16(Y)) return fail(QLORA_ERR_ALIGN, "X and Y must be 16-byte aligned");
+    if (U_save && !aligned16(U_save)) return fail(QLORA_ERR_ALIGN, "U_save must be 16-byte aligned");
+    if (M <= 0 || M > INT32_MAX) return fail(QLORA_ERR_SHAPE, "M (%lld) must be in [1, 2^31)", (long long)M);
+    QL_TRY(check_rank(r, scaling, A, B));
+    const int64_t N = w->n_out, K = w->n_in;
+    const WsLayout L = ws_layout(M, N, r, false);
+    QL_TRY(check_ws(ws, ws_bytes, L.total));
+    QL_TRY(require_sm100());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint16_t *us = reinterpret_cast<uint16_t *>(wsb);
+    if (r > 0)
+        QL_TRY(rank_side_product(true, X, M, K, A, r, scaling, us, reinterpret_cast<float *>(wsb + L.rank_bf16),
+                                 U_save, st));
+    // every M on CTA pairs (a small M pads the token tile)
+    return launch_fwd_pair(base_of_q8(w), X, M, N, K, B, r, us, Y, st);
+}
+
+qlora_status qlora_q8_0_lora_linear_bwd_dx(const qlora_q8_0_weight *w, const qlora_bf16 *dY, int64_t M,
+                                           const qlora_bf16 *A, const qlora_bf16 *B, int r, float scaling,
+                                           qlora_bf16 *dX, qlora_bf16 *G_save, void *ws, size_t ws_bytes,
+                                           void *stream) {
+    QL_TRY(check_q8(w));
+    if (!dY || !dX) return fail(QLORA_ERR_ARG, "dY and dX must be non-NULL");
+    if (!aligned16(dY) || !aligned16(dX)) return fail(QLORA_ERR_ALIGN, "dY and dX must be 16-byte aligned");
+    if (G_save && !aligned16(G_save)) return fail(QLORA_ERR_ALIGN, "G_save must be 16-byte aligned");
+    if (M <= 0 || M > INT32_MAX) return fail(QLORA_ERR_SHAPE, "M (%lld) must be in [1, 2^31)", (long long)M);
+    QL_TRY(check_rank(r, scaling, A, B));
+    const int64_t N = w->n_out, K = w->n_in;
+    if (N % 8) return fail(QLORA_ERR_SHAPE, "n_out (%lld) must be a multiple of 8 for the dX pass", (long long)N);
+    const DxPlan g = plan_dx(M, N, K);
+    const bool split = g.splits > 1;
+    const WsLayout L = ws_layout(M, K, r, split);
+    QL_TRY(check_ws(ws, ws_bytes, L.total));
+    QL_TRY(require_sm100());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    uint16_t *gs = reinterpret_cast<uint16_t *>(wsb);
+    float *dxacc = split ? reinterpret_cast<float *>(wsb + L.rank_bf16 + L.rank_acc) : nullptr;
+    if (r > 0)
+        QL_TRY(rank_side_product(false, dY, M, N, B, r, scaling, gs, reinterpret_cast<float *>(wsb + L.rank_bf16),
+                                 G_save, st));
+    if (dxacc) QL_TRY(cuda_check(cudaMemsetAsync(dxacc, 0, size_t(M) * K * 4, st), "zero split accumulator"));
+    return launch_dx_pair(base_of_q8(w), g, dY, M, N, K, A, r, gs, dX, dxacc, st);
 }
 
 qlora_status qlora_lora_grad_AB(const qlora_bf16 *X, const qlora_bf16 *dY, const qlora_bf16 *U, const qlora_bf16 *G,
