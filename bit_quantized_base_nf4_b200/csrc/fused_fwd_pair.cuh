@@ -55,6 +55,7 @@ struct Params {
     const uint16_t *Blora;   // [N, r] bf16 or nullptr
     uint16_t *Y;             // [M, N] bf16
     int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
+    int raster_mode, raster_group;   // tile order of the pairs (raster_tile)
     float level[16];
 };
 
@@ -88,8 +89,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();      // 0: even CTA (issues the MMAs), 1: its peer
-    const int n0 = blockIdx.x * BM;               // blockIdx.x = 2 * pair + rank
-    const int m0 = blockIdx.y * p.BN;
+    // this pair's tile: 256 W rows x BN tokens, in the L2-friendly order of raster_tile
+    int wt, tt;
+    raster_tile(blockIdx.y * (gridDim.x / 2) + (blockIdx.x >> 1), gridDim.x / 2, gridDim.y, p.raster_mode,
+                p.raster_group, wt, tt);
+    const int n0 = (2 * wt + int(rank)) * BM;
+    const int m0 = tt * p.BN;
     const int my_m0 = m0 + int(rank) * half_bn;
     const int KB = p.K / 64;                      // 64-K chunks of the base
     const int QM = (KB + 1) / 2;                  // main stages

@@ -337,6 +337,26 @@ __device__ __forceinline__ void codes4_to_bf16x2(uint32_t c, const LevelBytes &t
     w23 = __byte_perm(l, h, 0x7362);
 }
 
+// Tile order of a grid of CTA pairs over nw weight tiles x nt token tiles, from the pair's
+// launch index c (pairs start in increasing c).  The tiles go in bands that L2 keeps
+// while the band is worked: mode 0 takes bands of g weight tiles, weight tile fastest,
+// each band over all token tiles (the band's weight stays in L2, token tiles stream);
+// mode 1 takes bands of g token tiles, token tile fastest (the band's activations stay,
+// the weight streams once per band).  A bijection of [0, nw nt) onto the tiles.
+__device__ __forceinline__ void raster_tile(int c, int nw, int nt, int mode, int g, int &wt, int &tt) {
+    if (mode == 0) {
+        const int band = c / (g * nt), r = c - band * g * nt;
+        const int gs = min(g, nw - band * g);
+        wt = band * g + r % gs;
+        tt = r / gs;
+    } else {
+        const int band = c / (g * nw), r = c - band * g * nw;
+        const int gs = min(g, nt - band * g);
+        tt = band * g + r % gs;
+        wt = r / gs;
+    }
+}
+
 // ------------------------------------------------------------------ CTA pairs (cluster of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
