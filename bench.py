@@ -39,11 +39,18 @@ CSRC = os.path.join(ROOT, "bit_quantized_base_nf4_b200", "csrc")
 # launches of one step of the 70B layer, from one ncu capture each (profiles/), with a
 # hash of the kernel sources that capture ran; a source change makes the figure stale
 # and the bench then reports null
-KERNEL_TRAFFIC = {}
+KERNEL_TRAFFIC = {
+    # attention 127.2 + 51.0 MB, FFN up 1052.5 + 58.3 MB, FFN down 940.6 + 218.9 MB
+    "dx": {"bytes": 2448462848, "src_sha": "e27309de12477909"},
+    # attention 138.5 + 56.3 MB, FFN up 1936.1 + 268.8 MB, FFN down 1170.9 + 74.1 MB
+    "fwd": {"bytes": 3644764928, "src_sha": "fb65ee5cf55df8ee"},
+}
 
 
 def kernel_src_hash(kind: str) -> str:
-    files = {"dx": ["fused_bwd_pair.cuh", "ptx.cuh"], "fwd": ["fused_fwd_pair.cuh", "ptx.cuh"]}[kind]
+    # the kernel, its helpers, and the host code that picks its tiles and launch order
+    common = ["ptx.cuh", "scale_src.cuh", "qlora_nf4.cu"]
+    files = {"dx": ["fused_bwd_pair.cuh"] + common, "fwd": ["fused_fwd_pair.cuh"] + common}[kind]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(CSRC, f), "rb") as fh:
@@ -728,6 +735,8 @@ NCU_CASES = {
     "decode_m16": ([(4096, 4096)], 16, 8, "fwd"),
     "dx_70b_attn": ([(8192, 8192)], 4096, 0, "dx"),
     "fwd_70b_attn": ([(8192, 8192)], 4096, 0, "fwd"),
+    # the forward with the adapter: the rank-r product U = X A^T, then the GEMM
+    "fwd_r64_70b_attn": ([(8192, 8192)], 4096, 64, "fwd"),
     # the three matrices of the 70B layer, the GEMM kernel alone (r = 0) once each per step
     "dx_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "dx"),
     "fwd_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "fwd"),
