@@ -220,12 +220,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t a_off = h * 8192 + nl * 128;
         bool ok = true;
 
-        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
-        auto load_scale = [&](int s, float &qv, float &dv) {
+        // the raw scale words of this thread's 64-weight run in stage s (zero past the end);
+        // they are converted only when the stage is expanded, three group iterations later
+        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
             const int n = (nb_begin + s) * 64 + nl;
-            qv = 0.f;
+            qv = 0u;
             dv = 0.f;
-            if (!kQ8 && kvalid && s < NB && n < p.N) scale_parts(p.sc, int64_t(n) * KB + kblk, qv, dv);
+            if (!kQ8 && kvalid && s < NB && n < p.N) scale_load(p.sc, int64_t(n) * KB + kblk, qv, dv);
         };
         // Q8_0: the two fp16 scales of this thread's 64 weights of stage s (as one word)
         auto load_d8 = [&](int s) -> uint32_t {
@@ -235,7 +236,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         };
         uint32_t ua = load_d8(grp), ub = load_d8(grp + kGroups), uc = load_d8(grp + 2 * kGroups);
         // block scales of this group's next three stages
-        float qa, qb, qc;
+        uint32_t qa, qb, qc;
         float da, db, dc;
         load_scale(grp, qa, da);
         load_scale(grp + kGroups, qb, db);
@@ -270,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             } else if (s < NB) {
                 const int ci = s >> 2, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
-                const float sv = __fmul_rn(qa, da);
+                const float sv = scale_of(p.sc, qa, da);
                 qa = qb; da = db; qb = qc; db = dc;
                 load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);

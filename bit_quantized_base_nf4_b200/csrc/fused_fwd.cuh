@@ -199,14 +199,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cswz = row & 7;
         bool ok = true;
         const int64_t row_block0 = int64_t(n) * KB + kb_begin;
-        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
-        auto load_scale = [&](int s, float &qv, float &dv) {
-            qv = 0.f;
+        // the raw scale words of a 64-weight run (zero past the row end), converted only
+        // when the stage is expanded
+        auto load_scale = [&](int s, uint32_t &qv, float &dv) {
+            qv = 0u;
             dv = 0.f;
-            if (valid && s < nmain) scale_parts(p.sc, row_block0 + s, qv, dv);
+            if (valid && s < nmain) scale_load(p.sc, row_block0 + s, qv, dv);
         };
         // block scales of this group's next three stages (12 stages of lookahead)
-        float qa, qb, qc;
+        uint32_t qa, qb, qc;
         float da, db, dc;
         load_scale(grp, qa, da);
         load_scale(grp + kGroups, qb, db);
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t out[32];
             if (s < nmain) {
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
-                const float sv = __fmul_rn(qa, da);
+                const float sv = scale_of(p.sc, qa, da);
                 qa = qb; da = db; qb = qc; db = dc;
                 load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);

@@ -209,24 +209,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t cswz = row & 7;
         bool ok = true;
         const int64_t row_block0 = int64_t(n) * KB;
-        // the two factors of a 64-weight run's scale (s = fp32(qv * dv))
-        auto load_scale = [&](int kb, float &qv, float &dv) {
-            qv = 0.f;
+        // the raw scale words of a 64-weight run (zero past the row end)
+        auto load_scale = [&](int kb, uint32_t &av, float &dv) {
+            av = 0u;
             dv = 0.f;
-            if (!kQ8 && valid && kb < KB) scale_parts(p.sc, row_block0 + kb, qv, dv);
+            if (!kQ8 && valid && kb < KB) scale_load(p.sc, row_block0 + kb, av, dv);
         };
-        // block scales of this group's current and next stage (two 64-blocks each)
-        float qa0, qa1, qb0, qb1;
-        float da0, da1, db0, db1;
-        load_scale(2 * grp, qa0, da0);
-        load_scale(2 * grp + 1, qa1, da1);
-        load_scale(2 * (grp + kGroups), qb0, db0);
-        load_scale(2 * (grp + kGroups) + 1, qb1, db1);
+        // Q8_0: the four fp16 scales of a 128-K stage (two words)
+        auto load_d8 = [&](int q, uint32_t &w0, uint32_t &w1) {
+            w0 = 0u;
+            w1 = 0u;
+            if (kQ8 && valid && q < QM) {
+                const uint32_t *drow = reinterpret_cast<const uint32_t *>(p.d8 + int64_t(n) * (p.K / 32));
+                w0 = __ldg(drow + 2 * q);
+                if (2 * q + 1 < KB) w1 = __ldg(drow + 2 * q + 1);
+            }
+        };
+        // scales of this group's next stage, loaded one group iteration (four stages) ahead
+        uint32_t q0, q1, e0, e1;
+        float d0, d1;
+        load_scale(2 * grp, q0, d0);
+        load_scale(2 * grp + 1, q1, d1);
+        load_d8(grp, e0, e1);
 
         for (int q = grp; q < Q && ok; q += kGroups) {
             const int g = grp;
-            if (!mbar_wait_cluster(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
+            const uint32_t slot = tmem_a + lane_addr + g * 64;
+            // a main stage has two 64-K halves except an odd last one; the adapter stage
+            // has a second half only for r > 64
+            const bool two = q < QM ? 2 * q + 1 < KB : p.r > 64;
+            // TMEM slot g is free once the MMAs of stage q - 4 have completed.  The first
+            // half of the stage is expanded before this wait, the second while the first
+            // is stored, so the wait is followed by stores rather than by the whole expansion.
+            auto wait_slot = [&]() -> bool {
+                if (!mbar_wait_cluster(&free_b[g], ((q / kGroups) & 1) ^ 1, abort_flag)) return false;
+                tc_fence_after();
+                return true;
+            };
+            uint32_t out[32];
             if (kQ8 && q < QM) {
                 // Q8_0: this stage's 128 code bytes of the row and its four fp16 scales
                 const int sc = q % SC;
@@ -237,16 +257,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 8; ++i) cv[i] = lds128(cbase + ((uint32_t(i) ^ cswz) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c_empty[sc]);
-                uint32_t dpair[2] = {0u, 0u};
-                if (valid) {
-                    const uint32_t *drow = reinterpret_cast<const uint32_t *>(p.d8 + int64_t(n) * (p.K / 32));
-                    dpair[0] = __ldg(drow + 2 * q);
-                    if (2 * q + 1 < KB) dpair[1] = __ldg(drow + 2 * q + 1);
-                }
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    if (sub == 1 && 2 * q + 1 >= KB) break;   // odd last 64-K chunk
-                    uint32_t out[32];
+                const uint32_t dpair[2] = {e0, e1};
+                load_d8(q + kGroups, e0, e1);
+                auto expand = [&](int sub) {
                     const float d_lo = __half2float(__ushort_as_half(static_cast<unsigned short>(dpair[sub] & 0xFFFFu)));
                     const float d_hi = __half2float(__ushort_as_half(static_cast<unsigned short>(dpair[sub] >> 16)));
 #pragma unroll
@@ -258,7 +271,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         q8_word_to_bf16x2(c.z, d, out[8 * v + 4], out[8 * v + 5]);
                         q8_word_to_bf16x2(c.w, d, out[8 * v + 6], out[8 * v + 7]);
                     }
-                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                };
+                expand(0);
+                if (!wait_slot()) { ok = false; break; }
+                tmem_st32_checked(slot, out);
+                if (two) {
+                    expand(1);
+                    tmem_st32_checked(slot + 32, out);
                 }
             } else if (q < QM) {
                 const int ci = q >> 1, sc = ci % SC;
@@ -271,19 +290,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint4 c3 = lds128(cbase + (((jq + 3u) ^ cswz) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&c_empty[sc]);
-                const float sv0 = __fmul_rn(qa0, da0);
-                const float sv1 = __fmul_rn(qa1, da1);
-                qa0 = qb0; da0 = db0; qa1 = qb1; da1 = db1;
-                load_scale(2 * (q + 2 * kGroups), qb0, db0);
-                load_scale(2 * (q + 2 * kGroups) + 1, qb1, db1);
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    if (sub == 1 && 2 * q + 1 >= KB) break;   // odd last chunk
+                const float sv0 = scale_of(p.sc, q0, d0);
+                const float sv1 = scale_of(p.sc, q1, d1);
+                load_scale(2 * (q + kGroups), q0, d0);
+                load_scale(2 * (q + kGroups) + 1, q1, d1);
+                auto expand = [&](int sub) {
                     __nv_bfloat162 s2b = __float2bfloat162_rn(sub ? sv1 : sv0);
                     const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
                     const uint4 ca = sub ? c2 : c0, cb = sub ? c3 : c1;
                     const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
-                    uint32_t out[32];
                     // levels from the register byte tables (no shared-memory traffic)
 #pragma unroll
                     for (int w8 = 0; w8 < 8; ++w8) {
@@ -292,23 +307,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int by = 0; by < 4; ++by) out[w8 * 4 + by] = bf16x2_mul(out[w8 * 4 + by], s2);
                     }
-                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                };
+                expand(0);
+                if (!wait_slot()) { ok = false; break; }
+                tmem_st32_checked(slot, out);
+                if (two) {
+                    expand(1);
+                    tmem_st32_checked(slot + 32, out);
                 }
             } else {
                 // adapter stage: A operand = B_lora row n, elements 0 .. 127 (zero past r)
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    if (sub * 64 >= p.r) break;
-                    uint32_t out[32];
+                auto fill = [&](int sub) {
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
                         uint4 w = make_uint4(0, 0, 0, 0);
-                        const int e0 = sub * 64 + v * 8;
-                        if (valid && e0 < p.r)
-                            w = __ldg(reinterpret_cast<const uint4 *>(p.Blora + int64_t(n) * p.r + e0));
+                        const int e = sub * 64 + v * 8;
+                        if (valid && e < p.r)
+                            w = __ldg(reinterpret_cast<const uint4 *>(p.Blora + int64_t(n) * p.r + e));
                         out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
                     }
-                    tmem_st32_checked(tmem_a + lane_addr + g * 64 + sub * 32, out);
+                };
+                fill(0);
+                if (!wait_slot()) { ok = false; break; }
+                tmem_st32_checked(slot, out);
+                if (two) {
+                    fill(1);
+                    tmem_st32_checked(slot + 32, out);
                 }
             }
             tc_fence_before();

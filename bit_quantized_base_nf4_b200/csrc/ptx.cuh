@@ -480,14 +480,16 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
 __device__ __forceinline__ void tmem_st32_checked(uint32_t taddr, const uint32_t (&v)[32]) {
     tmem_st32(taddr, v);
     tmem_wait_st();
-    uint32_t r0[16], r1[16];
-    tmem_ld16(taddr, r0);
-    tmem_ld16(taddr + 16, r1);
-    tmem_wait_ld16(r0);
-    tmem_wait_ld16(r1);
+    // read back in two halves through one 16-register buffer (fewer live registers)
+    uint32_t r[16];
     uint32_t diff = 0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) diff |= (r0[e] ^ v[e]) | (r1[e] ^ v[16 + e]);
+    for (int h = 0; h < 2; ++h) {
+        tmem_ld16(taddr + 16 * h, r);
+        tmem_wait_ld16(r);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) diff |= r[e] ^ v[16 * h + e];
+    }
     if (diff) atomicExch(&g_device_error, kDeviceErrTmemStore);
 }
 

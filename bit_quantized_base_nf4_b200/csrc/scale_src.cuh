@@ -29,6 +29,24 @@ __device__ __forceinline__ void scale_parts(const ScaleSrc &s, int64_t b64, floa
     }
 }
 
+// The same two factors as raw loaded words: the u8 q_b (or the bits of the fp32 a_b) and
+// d_g (1 without double quantization).  Nothing here uses the loaded values, so a load
+// issued well ahead of its use does not wait for memory until scale_of runs.
+__device__ __forceinline__ void scale_load(const ScaleSrc &s, int64_t b64, uint32_t &a, float &d) {
+    const int64_t b = b64 >> s.blk_shift;
+    if (s.dq) {
+        a = __ldg(s.scales + b);
+        d = __ldg(s.scales2 + (b >> 8));
+    } else {
+        a = __ldg(reinterpret_cast<const uint32_t *>(s.scales) + b);
+        d = 1.f;
+    }
+}
+// s_b from the raw words of scale_load: fp32(q_b * d_g), or a_b itself
+__device__ __forceinline__ float scale_of(const ScaleSrc &s, uint32_t a, float d) {
+    return s.dq ? __fmul_rn(static_cast<float>(a), d) : __uint_as_float(a);
+}
+
 __device__ __forceinline__ float block_scale(const ScaleSrc &s, int64_t b64) {
     float sa, sb;
     scale_parts(s, b64, sa, sb);
