@@ -8,7 +8,10 @@
 // weight for its own 128 k into its own shared memory, as the MN-major
 // (k contiguous) 128-byte-swizzled A operand, and loads only its half of the
 // token tile (BN/2 rows of dY); one tcgen05.mma.cta_group::2 issued by the even
-// CTA reads both CTAs' A halves and B halves.
+// CTA reads both CTAs' A halves and B halves.  A 512-token tile uses two
+// accumulators of 256 columns (the whole TMEM), tokens 0..255 and 256..511: each
+// stage's A tile then feeds twice the MMA work, which halves the dequant, the A
+// stores and their fences per flop.
 //
 // The MMA issue is effectively synchronous with the issuing thread, so the MMA
 // thread does one barrier wait and one commit per stage of 64 n (four MMAs of
@@ -20,10 +23,11 @@
 //   producer (warp 3)    packed codes, 256 n rows x 128 k (four stages) per TMA
 //                        instruction
 //   dequant group s % 4  (4 warps, thread = one 64-block: a row n and a 64-k half)
-//                        expands the block through a byte -> (level[lo], level[hi])
-//                        bf16x2 table times the bf16 block scale, stores it
+//                        expands the block through the register level tables
+//                        (codes4_to_bf16x2) times the bf16 block scale, stores it
 //                        swizzled into A slot s % 4, then arrives on a_full
-//   MMA (warp 1, even)   four tcgen05.mma (K = 16), A and B from shared memory
+//   MMA (warp 1, even)   four tcgen05.mma (K = 16) per accumulator, A and B from
+//                        shared memory
 // Commits are multicast to both CTAs (free, acc_full); each CTA then reads back
 // its own 128 x BN accumulator and writes dX, or, when the contraction over n is
 // split across blockIdx.z (few output tiles: small M), adds it into an fp32
@@ -60,7 +64,7 @@ struct Params {
     const uint16_t *Alora;   // [r, K] bf16 or nullptr
     uint16_t *dX;            // [M, K] bf16 (one split)
     float *dXacc;            // [M, K] fp32 accumulator, zeroed by the host (several splits), or nullptr
-    int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32
+    int M, N, K, r, BN;      // BN: tokens per pair tile, a multiple of 32 up to 256, or 512
     int nb_per_split;        // 64-n stages per split along blockIdx.z (a multiple of 4)
     int raster_mode, raster_group;   // tile order of the pairs (raster_tile)
     float level[16];
@@ -70,7 +74,7 @@ __host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
     return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes * (q8 ? 2 : 1) + 512;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
-    return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u;
+    return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : BN <= 256 ? 256u : 512u;
 }
 
 template <bool kQ8>
@@ -82,6 +86,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int half_bn = p.BN / 2;
     const int ysb = half_bn * 128;                // this CTA's dY half for one stage
+    const int nacc = p.BN > 256 ? 2 : 1;          // accumulators of bna tokens each
+    const int bna = p.BN > 256 ? 256 : p.BN;
+    const int yab = (bna / 2) * 128;              // this CTA's share of one accumulator's dY, per stage
     uint8_t *sY = smem;
     uint8_t *sA = sY + S * ysb;
     uint8_t *sC = sA + S * kAStageBytes;
@@ -102,7 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 p.raster_group, wt, tt);
     const int k0 = (2 * wt + int(rank)) * BM;
     const int m0 = tt * p.BN;
-    const int my_m0 = m0 + int(rank) * half_bn;
+    const int my_m0 = m0 + int(rank) * (bna / 2);   // this CTA's tokens: my_m0 + 256 j + [0, bna / 2)
     const int KB = p.K / 64;
     const int NB_all = (p.N + 63) / 64;
     const int nb_begin = blockIdx.z * p.nb_per_split;          // first 64-n stage of this split
@@ -154,10 +161,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!mbar_wait_cluster(&free_b[sx], ((s / S) & 1) ^ 1, abort_flag)) break;
                 const uint32_t bar0 = mapa_shared(smem_u32(&y_full[sx]), 0);
                 if (rank == 0) mbar_arrive_expect_tx(&y_full[sx], 2 * ysb);
-                if (s < NB)
-                    tma_load_2d_pair(sY + sx * ysb, &tmY, bar0, (nb_begin + s) * 64, my_m0);
-                else
-                    tma_load_2d_pair(sY + sx * ysb, &tmG, bar0, (s - NB) * 64, my_m0);
+                for (int j = 0; j < nacc; ++j) {
+                    if (s < NB)
+                        tma_load_2d_pair(sY + sx * ysb + j * yab, &tmY, bar0, (nb_begin + s) * 64, my_m0 + 256 * j);
+                    else
+                        tma_load_2d_pair(sY + sx * ysb + j * yab, &tmG, bar0, (s - NB) * 64, my_m0 + 256 * j);
+                }
                 issued = s + 1;
             }
             // the even CTA sees both CTAs' copies complete on its barriers
@@ -185,7 +194,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer (even CTA only)
         if (lane == 0 && rank == 0) {
-            const uint32_t idesc = make_idesc_bf16(2 * BM, p.BN, 1, 0);
+            const uint32_t idesc = make_idesc_bf16(2 * BM, bna, 1, 0);
             for (int s = 0; s < total; ++s) {
                 const int g = s % S;
                 if (!mbar_wait_cluster(&a_full[g], (s / S) & 1, abort_flag)) break;
@@ -195,8 +204,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t abase = smem_u32(sA + g * kAStageBytes);
                 for (int kk = 0; kk < nk; ++kk) {
                     const uint64_t adesc = make_sdesc_sw128(abase + kk * 2048, 8192, 1024);
-                    const uint64_t bdesc = make_sdesc_sw128(ybase + kk * 32, 16, 1024);
-                    mma_ss_pair(tmem_acc, adesc, bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    for (int j = 0; j < nacc; ++j) {
+                        const uint64_t bdesc = make_sdesc_sw128(ybase + j * yab + kk * 32, 16, 1024);
+                        mma_ss_pair(tmem_acc + 256 * j, adesc, bdesc, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 tc_commit_pair(&free_b[g]);
             }

@@ -216,7 +216,12 @@ struct DxPlan {
     int64_t pairs, tiles_tok;
     int splits, nb_per_split;
 };
-DxPlan plan_dx(int64_t M, int64_t N, int64_t K) {
+// Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed, which
+// needs the shared memory of 4-bit codes.  They are taken when the estimated time of the
+// whole grid is lower: per pair tile about 0.62 us per 64-n stage at 256 tokens and about
+// 0.80 us at 512 (measured on the 70B shapes), plus about 10 us of set-up and epilogue,
+// times the number of waves of the pair tiles over the SM pairs.
+DxPlan plan_dx(int64_t M, int64_t N, int64_t K, bool wide) {
     DxPlan d;
     d.BN = pair_token_tile(M);
     d.pairs = ceil_div(K, 2 * bwdp::BM);
@@ -228,10 +233,18 @@ DxPlan plan_dx(int64_t M, int64_t N, int64_t K) {
     if (tiles * 2 <= pair_slots) splits = std::min(ceil_div(pair_slots, tiles), std::max<int64_t>(1, nb / 4));
     d.nb_per_split = static_cast<int>(ceil_div(ceil_div(nb, splits), 4) * 4);
     d.splits = static_cast<int>(ceil_div(nb, d.nb_per_split));
+    if (wide && d.splits == 1 && M > 256) {
+        const int64_t t512 = ceil_div(M, 512);
+        const double w256 = double(ceil_div(tiles, pair_slots)), w512 = double(ceil_div(d.pairs * t512, pair_slots));
+        if (w512 * (double(nb) * 0.80 + 10.0) < w256 * (double(nb) * 0.62 + 10.0)) {
+            d.BN = 512;
+            d.tiles_tok = t512;
+        }
+    }
     return d;
 }
 size_t bwd_ws_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    return ws_layout(M, K, r, plan_dx(M, N, K).splits > 1).total;
+    return ws_layout(M, K, r, plan_dx(M, N, K, false).splits > 1).total;
 }
 
 // Launches the rank-r tensor-core product out[i*ld_i + j*ld_j] += scaling *
@@ -409,8 +422,9 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
                             const qlora_bf16 *A, int r, const uint16_t *gs, qlora_bf16 *dX, float *dxacc,
                             cudaStream_t st) {
     const int BN = g.BN;
+    const int box = std::min(BN, 256) / 2;        // dY rows per TMA box: one CTA's share of an accumulator
     CUtensorMap tmY, tmC, tmG;
-    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN / 2, 64,
+    QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, box, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
     if (bw.q8)
         QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bwdp::kChunkRows, 128,
@@ -419,7 +433,7 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
         QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
                             CU_TENSOR_MAP_SWIZZLE_64B));
     if (r > 0)
-        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, BN / 2, 64,
+        QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, box, 64,
                             CU_TENSOR_MAP_SWIZZLE_128B));
     else
         tmG = tmY;
@@ -447,7 +461,7 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
         QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<true>, bwdp::smem_bytes(256, true)));
         bwdp::fused_bwd_pair_kernel<true><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN, true), st>>>(tmY, tmC, tmG, p);
     } else {
-        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<false>, bwdp::smem_bytes(256)));
+        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<false>, bwdp::smem_bytes(512)));
         bwdp::fused_bwd_pair_kernel<false><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
     }
     QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
@@ -766,7 +780,7 @@ qlora_status qlora_lora_linear_bwd_dx(const qlora_nf4_weight *w, const qlora_bf1
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     // CTA pairs at every M; split-K over n when the output tiles are few
-    const DxPlan g = plan_dx(M, N, K);
+    const DxPlan g = plan_dx(M, N, K, true);
     const bool split = g.splits > 1;
     const WsLayout L = ws_layout(M, K, r, split);
     uint8_t *wsb = static_cast<uint8_t *>(ws);
@@ -868,7 +882,7 @@ qlora_status qlora_q8_0_lora_linear_bwd_dx(const qlora_q8_0_weight *w, const qlo
     QL_TRY(check_rank(r, scaling, A, B));
     const int64_t N = w->n_out, K = w->n_in;
     if (N % 8) return fail(QLORA_ERR_SHAPE, "n_out (%lld) must be a multiple of 8 for the dX pass", (long long)N);
-    const DxPlan g = plan_dx(M, N, K);
+    const DxPlan g = plan_dx(M, N, K, false);
     const bool split = g.splits > 1;
     const WsLayout L = ws_layout(M, K, r, split);
     QL_TRY(check_ws(ws, ws_bytes, L.total));
