@@ -15,17 +15,19 @@
 //
 // The MMA issue is effectively synchronous with the issuing thread, so the MMA
 // thread does one barrier wait and one commit per stage of 64 n (four MMAs of
-// 256 x BN x 16): it waits on a_full[s % 4], which the even CTA's dequant warps
-// arrive on only after they have seen the stage's dY tile land, and commits to
-// free[s % 4], which releases the dY slot and the A slot of the stage in both CTAs.
+// 256 x BN x 16 per accumulator): it waits on a_full of the stage's slot s % kS,
+// which the even CTA's dequant warps arrive on only after they have seen the stage's
+// dY tile land, and commits to free[s % kS], which releases the dY slot and the A
+// slot of the stage in both CTAs.
 //   producer (warp 0)    one TMA instruction per stage: this CTA's dY half,
 //                        counted on the even CTA's y_full
-//   producer (warp 3)    packed codes, 256 n rows x 128 k (four stages) per TMA
+//   producer (warp 3)    packed codes, 64 kCS n rows x 128 k (kCS stages) per TMA
 //                        instruction
 //   dequant group s % 4  (4 warps, thread = one 64-block: a row n and a 64-k half)
+//                        expands the stage's weights ahead of its slot
 //                        expands the block through the register level tables
 //                        (codes4_to_bf16x2) times the bf16 block scale, stores it
-//                        swizzled into A slot s % 4, then arrives on a_full
+//                        swizzled into A slot s % kS, then arrives on a_full
 //   MMA (warp 1, even)   four tcgen05.mma (K = 16) per accumulator, A and B from
 //                        shared memory
 // Commits are multicast to both CTAs (free, acc_full); each CTA then reads back
@@ -48,13 +50,12 @@ namespace qlora {
 namespace bwdp {
 
 constexpr int BM = 128;                       // k columns of W0 per CTA (256 per pair)
-constexpr int S = 4;                          // stage slots: dY ring = A ring = dequant groups
-constexpr int kGroups = S;
-constexpr int SC = 2;                         // code ring chunks (four stages each)
-constexpr int kDqWarps = 4 * kGroups;
-constexpr int kThreads = 128 + 32 * kDqWarps;
-constexpr int kChunkRows = 256;               // n rows per code chunk
-constexpr int kCodeChunkBytes = kChunkRows * 64;   // 64 bytes = 128 k per row
+constexpr int SC = 2;                         // code ring chunks (kCS stages each)
+// kS stage slots (dY ring = A ring) and kS dequant groups of four warps: stage s goes to
+// slot and group s % kS, so that a group never reaches a slot's barriers a phase early.
+// A code chunk holds kCS stages (64 n rows each).
+__host__ __device__ constexpr int threads_for(int kS) { return 128 + 128 * kS; }
+__host__ __device__ constexpr int chunk_rows(int kCS) { return 64 * kCS; }
 constexpr int kAStageBytes = 64 * BM * 2;     // 64 n x 128 k bf16
 constexpr int kLutWords = 256 * 32;
 
@@ -70,18 +71,20 @@ struct Params {
     float level[16];
 };
 
-__host__ __device__ constexpr int smem_bytes(int BN, bool q8 = false) {
-    return 1024 + S * (BN / 2) * 128 + S * kAStageBytes + SC * kCodeChunkBytes * (q8 ? 2 : 1) + 512;
+// code rows of 64 (4-bit) or 128 (8-bit) bytes
+__host__ __device__ constexpr int smem_bytes(int BN, bool q8, int kS, int kCS) {
+    return 1024 + kS * (BN / 2) * 128 + kS * kAStageBytes + SC * chunk_rows(kCS) * (q8 ? 128 : 64) + 512;
 }
 __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
     return BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : BN <= 256 ? 256u : 512u;
 }
 
-template <bool kQ8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+template <bool kQ8, int kS, int kCS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
     fused_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmC,
                           const __grid_constant__ CUtensorMap tmG, const Params p) {
-    constexpr int kCB = kCodeChunkBytes * (kQ8 ? 2 : 1);   // 256 code rows of 64 (4-bit) or 128 (8-bit) bytes
+    constexpr int kGroups = kS;
+    constexpr int kCB = chunk_rows(kCS) * (kQ8 ? 128 : 64);   // one code chunk in shared memory
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int half_bn = p.BN / 2;
@@ -90,13 +93,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int bna = p.BN > 256 ? 256 : p.BN;
     const int yab = (bna / 2) * 128;              // this CTA's share of one accumulator's dY, per stage
     uint8_t *sY = smem;
-    uint8_t *sA = sY + S * ysb;
-    uint8_t *sC = sA + S * kAStageBytes;
+    uint8_t *sA = sY + kS * ysb;
+    uint8_t *sC = sA + kS * kAStageBytes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sC + SC * kCB);
-    uint64_t *y_full = bars, *free_b = bars + S;
-    uint64_t *c_full = bars + 2 * S, *c_empty = c_full + SC;
+    uint64_t *y_full = bars, *free_b = bars + kS;
+    uint64_t *c_full = bars + 2 * kS, *c_empty = c_full + SC;
     uint64_t *a_full = c_empty + SC;
-    uint64_t *acc_full = a_full + S;
+    uint64_t *acc_full = a_full + kS;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     float *s_level = reinterpret_cast<float *>(tmem_slot + 2);
@@ -117,7 +120,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // adapter stages (64 j each), on the last split only
     const int LS = (p.r > 0 && nb_begin + NB == NB_all) ? (p.r + 63) / 64 : 0;
     const int total = NB + LS;
-    const int nchunk = (NB + 3) / 4;
+    const int nchunk = (NB + kCS - 1) / kCS;
     const uint32_t ncols = tmem_cols(p.BN);
 
     if (threadIdx.x < 16) {
@@ -128,13 +131,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         s_level[threadIdx.x] = v;
     }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < S; ++i) {
+        for (int i = 0; i < kS; ++i) {
             mbar_init(&y_full[i], 1);
             mbar_init(&free_b[i], 1);
             mbar_init(&a_full[i], 8);             // 4 warps x 2 CTAs
         }
-        // a chunk is read by the four groups of its four stages
-        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 4 * kGroups); }
+        // a chunk is read by the groups of its kCS stages (four warps each)
+        for (int i = 0; i < SC; ++i) { mbar_init(&c_full[i], 1); mbar_init(&c_empty[i], 4 * kCS); }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -157,8 +160,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (LS) tma_prefetch_desc(&tmG);
             int issued = 0;
             for (int s = 0; s < total; ++s) {
-                const int sx = s % S;
-                if (!mbar_wait_cluster(&free_b[sx], ((s / S) & 1) ^ 1, abort_flag)) break;
+                const int sx = s % kS;
+                if (!mbar_wait_cluster(&free_b[sx], ((s / kS) & 1) ^ 1, abort_flag)) break;
                 const uint32_t bar0 = mapa_shared(smem_u32(&y_full[sx]), 0);
                 if (rank == 0) mbar_arrive_expect_tx(&y_full[sx], 2 * ysb);
                 for (int j = 0; j < nacc; ++j) {
@@ -171,10 +174,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             // the even CTA sees both CTAs' copies complete on its barriers
             if (rank == 0)
-                for (int s = max(0, issued - S); s < issued; ++s) mbar_drain(&y_full[s % S], (s / S) & 1);
+                for (int s = max(0, issued - kS); s < issued; ++s) mbar_drain(&y_full[s % kS], (s / kS) & 1);
             // producer tail: the release commits of the last stages land on this CTA's barriers
             // before it exits, so none can reach the shared memory of a CTA launched after it
-            for (int s = max(0, issued - S); s < issued; ++s) mbar_drain_cluster(&free_b[s % S], (s / S) & 1);
+            for (int s = max(0, issued - kS); s < issued; ++s) mbar_drain_cluster(&free_b[s % kS], (s / kS) & 1);
         }
     } else if (warp == 3) {
         // ---------------- packed-code producer (local to each CTA)
@@ -185,8 +188,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const int sc = c % SC;
                 if (!mbar_wait(&c_empty[sc], ((c / SC) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(&c_full[sc], kCB);
-                // rows n = 64 nb_begin + 256c .., bytes k0/2 .. k0/2 + 63 (4-bit) or k0 .. k0 + 127 (8-bit)
-                tma_load_2d(sC + sc * kCB, &tmC, &c_full[sc], kQ8 ? k0 : k0 / 2, nb_begin * 64 + c * kChunkRows);
+                // rows n = 64 (nb_begin + kCS c) .., bytes k0/2 .. k0/2 + 63 (4-bit) or k0 .. k0 + 127 (8-bit)
+                tma_load_2d(sC + sc * kCB, &tmC, &c_full[sc], kQ8 ? k0 : k0 / 2, nb_begin * 64 + c * chunk_rows(kCS));
                 issued = c + 1;
             }
             for (int c = max(0, issued - SC); c < issued; ++c) mbar_drain(&c_full[c % SC], (c / SC) & 1);
@@ -196,8 +199,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0 && rank == 0) {
             const uint32_t idesc = make_idesc_bf16(2 * BM, bna, 1, 0);
             for (int s = 0; s < total; ++s) {
-                const int g = s % S;
-                if (!mbar_wait_cluster(&a_full[g], (s / S) & 1, abort_flag)) break;
+                const int g = s % kS;
+                if (!mbar_wait_cluster(&a_full[g], (s / kS) & 1, abort_flag)) break;
                 tc_fence_after();
                 const int nk = (s < NB) ? 4 : min(4, (p.r - (s - NB) * 64 + 15) / 16);
                 const uint32_t ybase = smem_u32(sY + g * ysb);
@@ -254,16 +257,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         load_scale(grp + 2 * kGroups, qc, dc);
 
         for (int s = grp; s < total && ok; s += kGroups) {
-            const int g = grp;
+            const int g = s % kS;                   // stage slot
             uint32_t out[32];
             if (kQ8 && s < NB) {
-                const int ci = s >> 2, sc = ci % SC;
+                const int ci = s / kCS, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
                 const uint32_t dd = ua;
                 ua = ub; ub = uc;
                 uc = load_d8(s + 3 * kGroups);
                 // 128-byte code rows, 128-byte swizzle: 16-byte chunk j of row q sits at chunk j ^ (q & 7)
-                const uint32_t cbase = smem_u32(sC) + sc * kCB + ((s & 3) * 64 + nl) * 128;
+                const uint32_t cbase = smem_u32(sC) + sc * kCB + ((s % kCS) * 64 + nl) * 128;
                 uint4 cv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) cv[i] = lds128(cbase + (((4u * h + uint32_t(i)) ^ uint32_t(nl & 7)) << 4));
@@ -280,14 +283,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     q8_word_to_bf16x2(cv[v].w, d, out[8 * v + 6], out[8 * v + 7]);
                 }
             } else if (s < NB) {
-                const int ci = s >> 2, sc = ci % SC;
+                const int ci = s / kCS, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
                 const float sv = scale_of(p.sc, qa, da);
                 qa = qb; da = db; qb = qc; db = dc;
                 load_scale(s + 3 * kGroups, qc, dc);
                 __nv_bfloat162 s2b = __float2bfloat162_rn(sv);
                 const uint32_t s2 = *reinterpret_cast<uint32_t *>(&s2b);
-                const uint32_t cbase = smem_u32(sC) + sc * kCodeChunkBytes + ((s & 3) * 64 + nl) * 64;
+                const uint32_t cbase = smem_u32(sC) + sc * kCB + ((s % kCS) * 64 + nl) * 64;
                 const uint4 c0 = lds128(cbase + (((2u * h + 0u) ^ c_swz) << 4));
                 const uint4 c1 = lds128(cbase + (((2u * h + 1u) ^ c_swz) << 4));
                 __syncwarp();
@@ -313,8 +316,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     out[v * 4 + 0] = w.x; out[v * 4 + 1] = w.y; out[v * 4 + 2] = w.z; out[v * 4 + 3] = w.w;
                 }
             }
-            // A slot g is free once the MMAs of stage s - 4 have completed
-            if (!mbar_wait_cluster(&free_b[g], ((s / S) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            // A slot g is free once the MMAs of stage s - kS have completed
+            if (!mbar_wait_cluster(&free_b[g], ((s / kS) & 1) ^ 1, abort_flag)) { ok = false; break; }
             const uint32_t abase = sAu + g * kAStageBytes + a_off;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -324,7 +327,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             // the even CTA's warps arrive only once the stage's dY tile (both halves) has landed,
             // so a completed a_full also means a completed y_full for the MMA thread
-            if (rank == 0 && !mbar_wait_cluster(&y_full[g], (s / S) & 1, abort_flag)) { ok = false; break; }
+            if (rank == 0 && !mbar_wait_cluster(&y_full[g], (s / kS) & 1, abort_flag)) { ok = false; break; }
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
         }

@@ -216,11 +216,11 @@ struct DxPlan {
     int64_t pairs, tiles_tok;
     int splits, nb_per_split;
 };
-// Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed, which
-// needs the shared memory of 4-bit codes.  They are taken when the estimated time of the
-// whole grid is lower: per pair tile about 0.62 us per 64-n stage at 256 tokens and about
-// 0.80 us at 512 (measured on the 70B shapes), plus about 10 us of set-up and epilogue,
-// times the number of waves of the pair tiles over the SM pairs.
+// Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed (4-bit
+// codes only: 8-bit code chunks do not leave the shared memory for them).  They are taken
+// when the estimated time of the whole grid is lower: per pair tile about 0.73 us per
+// 64-n stage at 256 tokens and 1.03 us at 512 (measured on the 70B shapes), plus about
+// 10 us of set-up and epilogue, times the number of waves of the pair tiles over the SM pairs.
 DxPlan plan_dx(int64_t M, int64_t N, int64_t K, bool wide) {
     DxPlan d;
     d.BN = pair_token_tile(M);
@@ -236,7 +236,7 @@ DxPlan plan_dx(int64_t M, int64_t N, int64_t K, bool wide) {
     if (wide && d.splits == 1 && M > 256) {
         const int64_t t512 = ceil_div(M, 512);
         const double w256 = double(ceil_div(tiles, pair_slots)), w512 = double(ceil_div(d.pairs * t512, pair_slots));
-        if (w512 * (double(nb) * 0.80 + 10.0) < w256 * (double(nb) * 0.62 + 10.0)) {
+        if (w512 * (double(nb) * 1.03 + 10.0) < w256 * (double(nb) * 0.73 + 10.0)) {
             d.BN = 512;
             d.tiles_tok = t512;
         }
@@ -416,6 +416,22 @@ qlora_status launch_fwd_pair(const BaseW &bw, const qlora_bf16 *X, int64_t M, in
     return launch_check("fused_fwd_pair_kernel launch");
 }
 
+// The 512-token dX tiles run on three stage slots (= dequant groups) with four-stage code
+// chunks: 178 KB of shared memory.  Four slots (226 KB, or 210 KB with two-stage chunks)
+// returned a corrupted tile in up to 30 % of the calls on the 70B FFN shapes; three slots
+// and the 256-token tiles (165 KB) never did.
+constexpr int kDx512Slots = 3, kDx512ChunkStages = 4;
+
+template <bool kQ8, int kS, int kCS>
+qlora_status launch_dx_variant(dim3 grid, int BN, const CUtensorMap &tmY, const CUtensorMap &tmC,
+                               const CUtensorMap &tmG, const bwdp::Params &p, cudaStream_t st) {
+    const int most = kQ8 ? 256 : (kS == 4 && kCS == 4 ? 256 : 512);   // the largest tile this variant runs
+    QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>, bwdp::smem_bytes(most, kQ8, kS, kCS)));
+    bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>
+        <<<grid, bwdp::threads_for(kS), bwdp::smem_bytes(BN, kQ8, kS, kCS), st>>>(tmY, tmC, tmG, p);
+    return QLORA_OK;
+}
+
 // dX = dY W' + gs A on CTA pairs (gs = bf16(scaling * G) [M, r] in the workspace when
 // r > 0), split over n into dxacc (zeroed by the caller) when the plan says so.
 qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *dY, int64_t M, int64_t N, int64_t K,
@@ -426,11 +442,12 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     CUtensorMap tmY, tmC, tmG;
     QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, box, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
+    const int crow = bwdp::chunk_rows(BN > 256 && !bw.q8 ? kDx512ChunkStages : 4);   // code rows per TMA box
     if (bw.q8)
-        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, bwdp::kChunkRows, 128,
+        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, crow, 128,
                             CU_TENSOR_MAP_SWIZZLE_128B));
     else
-        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bwdp::kChunkRows, 64,
+        QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, crow, 64,
                             CU_TENSOR_MAP_SWIZZLE_64B));
     if (r > 0)
         QL_TRY(make_tmap_2d(&tmG, gs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, r, r, box, 64,
@@ -458,11 +475,11 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     for (int i = 0; i < 16; ++i) p.level[i] = bw.q8 ? 0.f : bw.level[i];
     dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
     if (bw.q8) {
-        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<true>, bwdp::smem_bytes(256, true)));
-        bwdp::fused_bwd_pair_kernel<true><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN, true), st>>>(tmY, tmC, tmG, p);
+        QL_TRY((launch_dx_variant<true, 4, 4>(grid, BN, tmY, tmC, tmG, p, st)));
+    } else if (BN > 256) {
+        QL_TRY((launch_dx_variant<false, kDx512Slots, kDx512ChunkStages>(grid, BN, tmY, tmC, tmG, p, st)));
     } else {
-        QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<false>, bwdp::smem_bytes(512)));
-        bwdp::fused_bwd_pair_kernel<false><<<grid, bwdp::kThreads, bwdp::smem_bytes(BN), st>>>(tmY, tmC, tmG, p);
+        QL_TRY((launch_dx_variant<false, 4, 4>(grid, BN, tmY, tmC, tmG, p, st)));
     }
     QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
     if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
