@@ -40,10 +40,10 @@ CSRC = os.path.join(ROOT, "bit_quantized_base_nf4_b200", "csrc")
 # hash of the kernel sources that capture ran; a source change makes the figure stale
 # and the bench then reports null
 KERNEL_TRAFFIC = {
-    # attention 127.2 + 51.0 MB, FFN up 1052.5 + 58.3 MB, FFN down 940.6 + 218.9 MB
-    "dx": {"bytes": 2448462848, "src_sha": "e27309de12477909"},
-    # attention 138.5 + 56.3 MB, FFN up 1936.1 + 268.8 MB, FFN down 1170.9 + 74.1 MB
-    "fwd": {"bytes": 3644764928, "src_sha": "fb65ee5cf55df8ee"},
+    # attention 170.1 + 47.1 MB, FFN up 852.0 + 58.8 MB, FFN down 893.5 + 212.0 MB
+    "dx": {"bytes": 2233458944, "src_sha": "5645f127b9703739"},
+    # attention 117.7 + 51.8 MB, FFN up 1951.7 + 221.4 MB, FFN down 1169.7 + 58.5 MB
+    "fwd": {"bytes": 3570799616, "src_sha": "5c58c99a5d9be592"},
 }
 
 
@@ -737,6 +737,8 @@ NCU_CASES = {
     "fwd_70b_attn": ([(8192, 8192)], 4096, 0, "fwd"),
     # the forward with the adapter: the rank-r product U = X A^T, then the GEMM
     "fwd_r64_70b_attn": ([(8192, 8192)], 4096, 64, "fwd"),
+    # the one-shot encode (fp32 -> NF4 + double quant) of the 8192 x 8192 matrix (268 MB in)
+    "encode_70b_attn": ([(8192, 8192)], 0, 0, "enc"),
     # the three matrices of the 70B layer, the GEMM kernel alone (r = 0) once each per step
     "dx_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "dx"),
     "fwd_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "fwd"),
@@ -745,13 +747,27 @@ NCU_CASES = {
 
 def ncu_case(name, steps, warmup):
     """A small, fixed launch sequence for profiler captures: per step, one call of one kind
-    (the forward or dX) on each listed matrix, nothing else after the setup."""
+    (the forward, dX or the one-shot encode) on each listed matrix, nothing else after the setup."""
     import torch
     import bit_quantized_base_nf4_b200 as q
     from bit_quantized_base_nf4_b200 import synthetic as syn
     shapes, M, r, kind = NCU_CASES[name]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if kind == "enc":
+        g = torch.Generator(device=dev)
+        g.manual_seed(5100)
+        encs = []
+        for N, K in shapes:
+            W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32) * 0.015
+            encs.append((W, q.NF4Weight.empty(N, K, device=dev)))
+        for _ in range(warmup + steps):
+            for W, w in encs:
+                q.qlora_quantize_nf4_dq(W, w)
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status()
+        print(json.dumps({"ncu_case": name, "calls": (warmup + steps) * len(encs)}), flush=True)
+        return
     runs = []
     for i, (N, K) in enumerate(shapes):
         c = syn.LayerCase(f"{name}-{i}", M=M, N=N, K=K, r=r, alpha=2.0 * r, w_std=0.015, seed=7000 + 10 * i)
