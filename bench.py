@@ -739,6 +739,8 @@ NCU_CASES = {
     "fwd_r64_70b_attn": ([(8192, 8192)], 4096, 64, "fwd"),
     # the one-shot encode (fp32 -> NF4 + double quant) of the 8192 x 8192 matrix (268 MB in)
     "encode_70b_attn": ([(8192, 8192)], 0, 0, "enc"),
+    # LoRA merge + requantize of the 8192 x 8192 matrix, r = 64 (merge kernel, then the encode)
+    "merge_70b_attn": ([(8192, 8192)], 0, 64, "merge"),
     # the three matrices of the 70B layer, the GEMM kernel alone (r = 0) once each per step
     "dx_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "dx"),
     "fwd_70b_layer": ([(8192, 8192), (28672, 8192), (8192, 28672)], 4096, 0, "fwd"),
@@ -747,13 +749,32 @@ NCU_CASES = {
 
 def ncu_case(name, steps, warmup):
     """A small, fixed launch sequence for profiler captures: per step, one call of one kind
-    (the forward, dX or the one-shot encode) on each listed matrix, nothing else after the setup."""
+    (the forward, dX, the one-shot encode or the merge) on each listed matrix, nothing else
+    after the setup."""
     import torch
     import bit_quantized_base_nf4_b200 as q
     from bit_quantized_base_nf4_b200 import synthetic as syn
     shapes, M, r, kind = NCU_CASES[name]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if kind == "merge":
+        g = torch.Generator(device=dev)
+        g.manual_seed(5200 + r)
+        merges = []
+        for N, K in shapes:
+            W = torch.randn(N, K, generator=g, device=dev, dtype=torch.float32) * 0.015
+            w = q.NF4Weight.empty(N, K, device=dev)
+            q.qlora_quantize_nf4_dq(W, w)
+            A = syn.normal_bf16((r, K), 1.0 / K, 5300 + r).to(dev)
+            B = syn.normal_bf16((N, r), 0.01, 5400 + r).to(dev)
+            merges.append((w, A, B, W, q.NF4Weight.empty(N, K, device=dev)))
+        for _ in range(warmup + steps):
+            for w, A, B, scratch, w_out in merges:
+                q.qlora_lora_merge_requant(w, A, B, r, 16.0 / r, scratch, w_out)
+        torch.cuda.synchronize(dev)
+        q.qlora_sync_status()
+        print(json.dumps({"ncu_case": name, "calls": (warmup + steps) * len(merges)}), flush=True)
+        return
     if kind == "enc":
         g = torch.Generator(device=dev)
         g.manual_seed(5100)

@@ -33,7 +33,7 @@ def flush():
     return torch.empty(256 << 20, dtype=torch.uint8, device=DEV)
 
 
-def _inputs(N, K, r, seed):
+def _inputs(N, K, r, seed, M=M):
     g = torch.Generator(device=DEV)
     g.manual_seed(seed)
     w = q.NF4Weight.empty(N, K)
@@ -82,3 +82,13 @@ def test_fwd_repeats_bit_exact(N, K, r, flush):
     out = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
     _repeat(lambda o: q.qlora_lora_linear_fwd(w, X, A, B, r, 2.0 if r else 0.0, o, None, ws), out, CALLS_FWD, flush,
             exact=r == 0)
+
+
+@pytest.mark.parametrize("N,K,m", [(4096, 11008, 1), (11008, 4096, 16), (4096, 4096, 4)])
+def test_small_m_forward_repeats_bit_exact(N, K, m, flush):
+    """The small-M forward keeps every partial sum in its CTA (the adapter's U included), so
+    its results are exact repeats too."""
+    r = 8
+    w, X, dY, A, B, ws = _inputs(N, K, r, 13, M=m)
+    out = torch.empty(m, N, dtype=torch.bfloat16, device=DEV)
+    _repeat(lambda o: q.qlora_lora_linear_fwd(w, X, A, B, r, 2.0, o, None, ws), out, CALLS_FWD, flush, exact=True)
