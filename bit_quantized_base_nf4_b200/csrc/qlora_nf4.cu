@@ -637,11 +637,12 @@ qlora_status qlora_lora_merge_requant(const qlora_nf4_weight *w_in, const qlora_
     if (!W_scratch) return fail(QLORA_ERR_ARG, "W_scratch is NULL");
     if (!aligned16(W_scratch)) return fail(QLORA_ERR_ALIGN, "W_scratch must be 16-byte aligned");
     QL_TRY(require_sm100());
-    // x: the code words of a row (8 weights each); y: rows, about 16 CTAs per SM in all
-    const int64_t gx = std::min<int64_t>(ceil_div(w_in->n_in / 8, 256), 32);
-    const int64_t gy = std::min<int64_t>(w_in->n_out, std::max<int64_t>(1, int64_t(sm_count()) * 16 / gx));
+    // x: a row's groups of kMergeCols weights; y: groups of kMergeRows rows, about 8 CTAs per SM in all
+    const int64_t gx = std::min<int64_t>(ceil_div(w_in->n_in / kMergeCols, kMergeThreads), 32);
+    const int64_t gy = std::min<int64_t>(ceil_div(w_in->n_out, kMergeRows),
+                                         std::max<int64_t>(1, int64_t(sm_count()) * 8 / gx));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    nf4_lora_merge_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
+    nf4_lora_merge_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), kMergeThreads, 0, st>>>(
         w_in->codes, scale_src(w_in), r > 0 ? reinterpret_cast<const uint16_t *>(A) : nullptr,
         r > 0 ? reinterpret_cast<const uint16_t *>(B) : nullptr, r, r > 0 ? scaling : 0.f, w_in->n_out, w_in->n_in,
         W_scratch, codebook_arg(w_in->quant_type));

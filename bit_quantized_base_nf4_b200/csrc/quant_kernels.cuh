@@ -247,56 +247,80 @@ __global__ void __launch_bounds__(256) q8_0_dequant_kernel(const int8_t *__restr
     }
 }
 
-// LoRA merge, the step before requantization.  Rows run over blockIdx.y, the row's
-// code words over x; a thread handles 8 weights (one code word).
+// LoRA merge, the step before requantization.
 //   m = bf16(RN32(bf16(w') + s * sum_j B[n, j] A[j, k])):
 // the dequantized base in bf16, the adapter product and the add in fp64 with j
-// ascending and no fused multiply-add (bf16 x bf16 products are exact in fp64), then
-// float32 and bf16 rounding.  m is stored as float32, the input of the encode kernel.
+// ascending, then float32 and bf16 rounding; m is stored as float32, the input of the
+// encode kernel.  A bf16 x bf16 product is exact in fp64 (16 significant bits, and the
+// exponent range of fp64 holds every such product), so the fused multiply-add
+// RN(acc + b a) used here equals the separate product and sum.
+// A thread takes kMergeCols consecutive weights of kMergeRows rows: each A value it
+// loads and widens serves every row, and B of the CTA's rows sits in shared memory as
+// fp64.  Rows run over blockIdx.y (in groups of kMergeRows), weights over x.
+constexpr int kMergeRows = 4, kMergeCols = 4, kMergeThreads = 256, kMergeMaxR = 128;
 __device__ __forceinline__ float merge_one(float level, float s, double sd, double acc) {
     const float wb = __bfloat162float(__float2bfloat16_rn(__fmul_rn(level, s)));
     const double t = __dadd_rn(static_cast<double>(wb), __dmul_rn(sd, acc));
     return __bfloat162float(__float2bfloat16_rn(__double2float_rn(t)));
 }
-__global__ void __launch_bounds__(256) nf4_lora_merge_kernel(const uint8_t *__restrict__ codes, const ScaleSrc sc,
-                                                             const uint16_t *__restrict__ A,
-                                                             const uint16_t *__restrict__ B, int r, float scaling,
-                                                             int64_t N, int64_t K, float *__restrict__ out,
-                                                             const CodebookArg cb) {
+__global__ void __launch_bounds__(kMergeThreads) nf4_lora_merge_kernel(const uint8_t *__restrict__ codes,
+                                                                       const ScaleSrc sc,
+                                                                       const uint16_t *__restrict__ A,
+                                                                       const uint16_t *__restrict__ B, int r,
+                                                                       float scaling, int64_t N, int64_t K,
+                                                                       float *__restrict__ out,
+                                                                       const CodebookArg cb) {
     __shared__ float s_lv[16];
+    __shared__ double s_b[kMergeRows][kMergeMaxR];
     float lv = 0.f;
 #pragma unroll
     for (int l = 0; l < 16; ++l)   // constant indices keep the parameter block out of local memory
         if ((threadIdx.x & 15) == l) lv = cb.level[l];
     if (threadIdx.x < 16) s_lv[threadIdx.x] = lv;
-    __syncthreads();
     const double sd = static_cast<double>(scaling);
-    const int64_t K8 = K / 8;
-    for (int64_t n = blockIdx.y; n < N; n += gridDim.y) {
-        for (int64_t c = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; c < K8; c += int64_t(gridDim.x) * blockDim.x) {
-            const int64_t i = n * K8 + c;   // code word index; 8 weights per word, 64 per block
-            const int64_t k0 = 8 * c;
-            const uint32_t cw = __ldg(reinterpret_cast<const uint32_t *>(codes) + i);
-            const float s = block_scale(sc, i >> 3);
-            double acc[8];
+    const int64_t KC = K / kMergeCols;            // column groups of a row
+    for (int64_t n0 = int64_t(blockIdx.y) * kMergeRows; n0 < N; n0 += int64_t(gridDim.y) * kMergeRows) {
+        __syncthreads();   // the previous row group is done with s_b
+        for (int t = threadIdx.x; t < kMergeRows * r; t += blockDim.x) {
+            const int rr = t / r, j = t - rr * r;
+            const int64_t n = n0 + rr;
+            s_b[rr][j] = n < N ? static_cast<double>(__uint_as_float(uint32_t(__ldg(B + n * r + j)) << 16)) : 0.0;
+        }
+        __syncthreads();
+        for (int64_t c = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; c < KC; c += int64_t(gridDim.x) * blockDim.x) {
+            const int64_t k0 = kMergeCols * c;
+            double acc[kMergeRows][kMergeCols];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+            for (int rr = 0; rr < kMergeRows; ++rr)
+#pragma unroll
+                for (int e = 0; e < kMergeCols; ++e) acc[rr][e] = 0.0;
             for (int j = 0; j < r; ++j) {
-                const double b = static_cast<double>(__uint_as_float(uint32_t(__ldg(B + n * r + j)) << 16));
-                const uint4 av = __ldg(reinterpret_cast<const uint4 *>(A + int64_t(j) * K + k0));
+                const uint2 av = __ldg(reinterpret_cast<const uint2 *>(A + int64_t(j) * K + k0));
+                const double a0 = static_cast<double>(__uint_as_float(av.x << 16));
+                const double a1 = static_cast<double>(__uint_as_float(av.x & 0xFFFF0000u));
+                const double a2 = static_cast<double>(__uint_as_float(av.y << 16));
+                const double a3 = static_cast<double>(__uint_as_float(av.y & 0xFFFF0000u));
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint32_t word = (e >> 1) == 0 ? av.x : (e >> 1) == 1 ? av.y : (e >> 1) == 2 ? av.z : av.w;
-                    const float a = __uint_as_float((e & 1) ? (word & 0xFFFF0000u) : (word << 16));
-                    acc[e] = __dadd_rn(acc[e], __dmul_rn(b, static_cast<double>(a)));
+                for (int rr = 0; rr < kMergeRows; ++rr) {
+                    const double b = s_b[rr][j];
+                    acc[rr][0] = __fma_rn(b, a0, acc[rr][0]);
+                    acc[rr][1] = __fma_rn(b, a1, acc[rr][1]);
+                    acc[rr][2] = __fma_rn(b, a2, acc[rr][2]);
+                    acc[rr][3] = __fma_rn(b, a3, acc[rr][3]);
                 }
             }
-            float m[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m[e] = merge_one(s_lv[(cw >> (4 * e)) & 15u], s, sd, acc[e]);
-            float4 *o = reinterpret_cast<float4 *>(out) + 2 * i;
-            o[0] = make_float4(m[0], m[1], m[2], m[3]);
-            o[1] = make_float4(m[4], m[5], m[6], m[7]);
+            for (int rr = 0; rr < kMergeRows; ++rr) {
+                const int64_t n = n0 + rr;
+                if (n >= N) break;
+                const int64_t w0 = n * K + k0;                          // first weight of the group
+                const uint32_t cw = __ldg(reinterpret_cast<const uint16_t *>(codes) + w0 / 4);   // 4 codes
+                const float s = block_scale(sc, w0 >> 6);
+                float m[kMergeCols];
+#pragma unroll
+                for (int e = 0; e < kMergeCols; ++e) m[e] = merge_one(s_lv[(cw >> (4 * e)) & 15u], s, sd, acc[rr][e]);
+                reinterpret_cast<float4 *>(out)[w0 / 4] = make_float4(m[0], m[1], m[2], m[3]);
+            }
         }
     }
 }
