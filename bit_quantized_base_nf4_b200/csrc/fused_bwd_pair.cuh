@@ -82,8 +82,15 @@ __host__ __device__ constexpr uint32_t tmem_cols(int BN) {
 template <bool kQ8, int kS, int kCS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
     fused_bwd_pair_kernel(const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmC,
-                          const __grid_constant__ CUtensorMap tmG, const Params p) {
+                          const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmD,
+                          const Params p) {
     constexpr int kGroups = kS;
+    // Group g reads code chunk s / kCS of each stage s = g (mod kS) and waits on its slot's
+    // c_full by parity.  A parity wait is only sound when the waiter saw the slot's
+    // previous phase complete, so every group must read every chunk: kCS >= kS.  (With
+    // two-stage chunks and three groups a group skips a chunk, and its next wait on that
+    // slot could pass while the skipped chunk was still in flight.)
+    static_assert(kCS >= kS, "every dequant group must read every code chunk");
     constexpr int kCB = chunk_rows(kCS) * (kQ8 ? 128 : 64);   // one code chunk in shared memory
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -270,8 +277,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
                 uint4 cv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) cv[i] = lds128(cbase + (((4u * h + uint32_t(i)) ^ uint32_t(nl & 7)) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const float d_lo = __half2float(__ushort_as_half(static_cast<unsigned short>(dd & 0xFFFFu)));
                 const float d_hi = __half2float(__ushort_as_half(static_cast<unsigned short>(dd >> 16)));
 #pragma unroll
@@ -282,6 +287,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
                     q8_word_to_bf16x2(cv[v].z, d, out[8 * v + 4], out[8 * v + 5]);
                     q8_word_to_bf16x2(cv[v].w, d, out[8 * v + 6], out[8 * v + 7]);
                 }
+                // released only once every code of the chunk this thread read has been used: a
+                // release right after the loads let the next copy overwrite codes still being read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
             } else if (s < NB) {
                 const int ci = s / kCS, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
@@ -293,8 +302,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
                 const uint32_t cbase = smem_u32(sC) + sc * kCB + ((s % kCS) * 64 + nl) * 64;
                 const uint4 c0 = lds128(cbase + (((2u * h + 0u) ^ c_swz) << 4));
                 const uint4 c1 = lds128(cbase + (((2u * h + 1u) ^ c_swz) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
                 // levels from the register byte tables (no shared-memory traffic)
 #pragma unroll
@@ -304,6 +311,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
 #pragma unroll
                     for (int by = 0; by < 4; ++by) out[w8 * 4 + by] = bf16x2_mul(out[w8 * 4 + by], s2);
                 }
+                // released only once every code of the chunk this thread read has been used: a
+                // release right after the loads let the next copy overwrite codes still being read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
             } else {
                 // adapter chunk: row j of A [r, K], 64 k starting at k0 + 64h (zero past r / K)
                 const int j = (s - NB) * 64 + nl;
@@ -333,32 +344,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_for(kS), 1)
         }
 
         // ---------------- epilogue: this CTA's 128 k rows x BN tokens
-        if (ok && mbar_wait_cluster(acc_full, 0, abort_flag)) {
+        const bool have = ok && mbar_wait_cluster(acc_full, 0, abort_flag);
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int k = k0 + row;
+        const uint32_t lane_addr = uint32_t(quad * 32) << 16;
+        const int nchunks = p.BN / 16;
+        if (have) {
             tc_fence_after();
-            const int quad = warp & 3;
-            const int row = quad * 32 + lane;
-            const int k = k0 + row;
-            const uint32_t lane_addr = uint32_t(quad * 32) << 16;
-            const int nchunks = p.BN / 16;
-            for (int ch = grp; ch < nchunks; ch += kGroups) {
-                uint32_t v[16];
-                tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
-                tmem_wait_ld16(v);
-                if (k < p.K) {
-                    const int mb = m0 + ch * 16;
-                    if (p.dXacc) {
+            if (p.dXacc) {
+                for (int ch = grp; ch < nchunks; ch += kGroups) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
+                    tmem_wait_ld16(v);
+                    if (k < p.K) {
+                        const int mb = m0 + ch * 16;
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             if (mb + i < p.M) atomicAdd(p.dXacc + int64_t(mb + i) * p.K + k, __uint_as_float(v[i]));
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (mb + i < p.M) {
-                                __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
-                                p.dX[int64_t(mb + i) * p.K + k] = *reinterpret_cast<uint16_t *>(&hv);
-                            }
                     }
                 }
+            } else {
+                // bf16 tile [token][128 k] in the ring memory, idle once the last MMAs completed
+                const uint32_t stage = smem_u32(smem);
+                for (int ch = grp; ch < nchunks; ch += kGroups) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
+                    tmem_wait_ld16(v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat16 hv = __float2bfloat16_rn(__uint_as_float(v[i]));
+                        sts16(stage + uint32_t(((ch * 16 + i) * BM + row) * 2), *reinterpret_cast<uint16_t *>(&hv));
+                    }
+                }
+            }
+        }
+        if (!p.dXacc) {
+            // every dequant warp passes here once, with or without a tile; one thread then
+            // stores the tile with TMA (the map clips tokens past M and columns past K)
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128 * kS);
+            if (dw == 0 && lane == 0 && have && *abort_flag == 0) {
+                for (int h = 0; h * 256 < p.BN; ++h)
+                    tma_store_2d(&tmD, smem + h * 256 * BM * 2, k0, m0 + 256 * h);
+                bulk_commit_group();
+                bulk_wait_all();
             }
         }
     }

@@ -227,8 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t j0 = 2u * uint32_t(s & 3);
                 const uint4 c0 = lds128(cbase + (((j0 + 0u) ^ cswz) << 4));
                 const uint4 c1 = lds128(cbase + (((j0 + 1u) ^ cswz) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                 for (int w8 = 0; w8 < 8; ++w8) {
@@ -238,6 +236,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         out[w8 * 4 + by] = bf16x2_mul(lds32_const(lut + (e << 7)), s2);
                     }
                 }
+                // released only once every code this thread read has been used: a release right
+                // after the loads let the next copy overwrite codes still being read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
             } else {
                 // adapter chunk: A operand = B_lora row n, elements e0 .. e0+63 (zero past r)
                 const int e0 = (s - nmain) * 64;

@@ -68,7 +68,8 @@ __host__ __device__ constexpr uint32_t tmem_cols(int) { return 512u; }
 template <bool kQ8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     fused_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmC,
-                          const __grid_constant__ CUtensorMap tmU, const Params p) {
+                          const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmY,
+                          const Params p) {
     constexpr int kStagesPerChunk = kQ8 ? 1 : 2;   // a 128-byte code row holds 256 (4-bit) or 128 (8-bit) K
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -255,8 +256,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 uint4 cv[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) cv[i] = lds128(cbase + ((uint32_t(i) ^ cswz) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const uint32_t dpair[2] = {e0, e1};
                 load_d8(q + kGroups, e0, e1);
                 auto expand = [&](int sub) {
@@ -279,6 +278,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     expand(1);
                     tmem_st32_checked(slot + 32, out);
                 }
+                // released only once every code of the chunk this thread read has been used: a
+                // release right after the loads let the next copy overwrite codes still being read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
             } else if (q < QM) {
                 const int ci = q >> 1, sc = ci % SC;
                 if (!mbar_wait(&c_full[sc], (ci / SC) & 1, abort_flag)) { ok = false; break; }
@@ -288,8 +291,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint4 c1 = lds128(cbase + (((jq + 1u) ^ cswz) << 4));
                 const uint4 c2 = lds128(cbase + (((jq + 2u) ^ cswz) << 4));
                 const uint4 c3 = lds128(cbase + (((jq + 3u) ^ cswz) << 4));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&c_empty[sc]);
                 const float sv0 = scale_of(p.sc, q0, d0);
                 const float sv1 = scale_of(p.sc, q1, d1);
                 load_scale(2 * (q + kGroups), q0, d0);
@@ -315,6 +316,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     expand(1);
                     tmem_st32_checked(slot + 32, out);
                 }
+                // released only once every code of the chunk this thread read has been used: a
+                // release right after the loads let the next copy overwrite codes still being read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
             } else {
                 // adapter stage: A operand = B_lora row n, elements 0 .. 127 (zero past r)
                 auto fill = [&](int sub) {
@@ -343,24 +348,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&a_full[g]), 0));
         }
 
-        // ---------------- epilogue: this CTA's 128 rows x BN tokens
-        if (ok && mbar_wait_cluster(acc_full, 0, abort_flag)) {
+        // ---------------- epilogue: this CTA's 128 rows x BN tokens, staged as a bf16
+        // [token][128 n] tile in the X ring (idle once the last MMAs completed), then one
+        // TMA store (the map clips tokens past M and rows past N)
+        const bool have = ok && mbar_wait_cluster(acc_full, 0, abort_flag);
+        if (have) {
             tc_fence_after();
+            const uint32_t stage = smem_u32(sX);
             const int nchunks = p.BN / 16;
             for (int ch = grp; ch < nchunks; ch += kGroups) {
                 uint32_t v[16];
                 tmem_ld16(tmem_acc + lane_addr + ch * 16, v);
                 tmem_wait_ld16(v);
-                if (valid) {
-                    const int mb = m0 + ch * 16;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (mb + i < p.M) {
-                            __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
-                            p.Y[int64_t(mb + i) * p.N + n] = *reinterpret_cast<uint16_t *>(&h);
-                        }
+                for (int i = 0; i < 16; ++i) {
+                    __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+                    sts16(stage + uint32_t(((ch * 16 + i) * BM + row) * 2), *reinterpret_cast<uint16_t *>(&h));
                 }
             }
+        }
+        // every dequant warp passes here once, with or without a tile
+        fence_proxy_async_smem();
+        named_bar_sync(1, 32 * kDqWarps);
+        if (dw == 0 && lane == 0 && have && *abort_flag == 0) {
+            tma_store_2d(&tmY, sX, n0, m0);
+            bulk_commit_group();
+            bulk_wait_all();
         }
     }
 

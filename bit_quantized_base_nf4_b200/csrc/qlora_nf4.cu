@@ -217,7 +217,7 @@ struct DxPlan {
     int splits, nb_per_split;
 };
 // Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed (4-bit
-// codes only: 8-bit code chunks do not leave the shared memory for them).  They are taken
+// codes only; see kDx512Slots).  They are taken
 // when the estimated time of the whole grid is lower: per pair tile about 0.73 us per
 // 64-n stage at 256 tokens and 1.03 us at 512 (measured on the 70B shapes), plus about
 // 10 us of set-up and epilogue, times the number of waves of the pair tiles over the SM pairs.
@@ -389,6 +389,10 @@ qlora_status launch_fwd_pair(const BaseW &bw, const qlora_bf16 *X, int64_t M, in
                             CU_TENSOR_MAP_SWIZZLE_128B));
     else
         tmU = tmX;
+    // the Y tile store of each CTA: [BN tokens, 128 rows of W] boxes, unswizzled
+    CUtensorMap tmY;
+    QL_TRY(make_tmap_2d(&tmY, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, BN, fwdp::BM,
+                        CU_TENSOR_MAP_SWIZZLE_NONE));
     fwdp::Params p;
     p.sc = bw.sc;
     p.d8 = bw.d8;
@@ -408,27 +412,30 @@ qlora_status launch_fwd_pair(const BaseW &bw, const qlora_bf16 *X, int64_t M, in
     dim3 grid(static_cast<unsigned>(2 * nw), static_cast<unsigned>(nt), 1);
     if (bw.q8) {
         QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel<true>, fwdp::smem_bytes(256, true)));
-        fwdp::fused_fwd_pair_kernel<true><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN, true), st>>>(tmX, tmC, tmU, p);
+        fwdp::fused_fwd_pair_kernel<true><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN, true), st>>>(tmX, tmC, tmU, tmY, p);
     } else {
         QL_TRY(set_smem(fwdp::fused_fwd_pair_kernel<false>, fwdp::smem_bytes(256)));
-        fwdp::fused_fwd_pair_kernel<false><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN), st>>>(tmX, tmC, tmU, p);
+        fwdp::fused_fwd_pair_kernel<false><<<grid, fwdp::kThreads, fwdp::smem_bytes(BN), st>>>(tmX, tmC, tmU, tmY, p);
     }
     return launch_check("fused_fwd_pair_kernel launch");
 }
 
-// The 512-token dX tiles run on three stage slots (= dequant groups) with four-stage code
-// chunks: 178 KB of shared memory.  Four slots (226 KB, or 210 KB with two-stage chunks)
-// returned a corrupted tile in up to 30 % of the calls on the 70B FFN shapes; three slots
-// and the 256-token tiles (165 KB) never did.
-constexpr int kDx512Slots = 3, kDx512ChunkStages = 4;
+// dX kernel forms, by shared memory: 4-bit codes take 256-token tiles on four stage
+// slots (= dequant groups) and four-stage code chunks (165 KB), or 512-token tiles on
+// three slots and four-stage chunks (178 KB); 8-bit codes take 256-token tiles on three
+// slots and three-stage chunks (146 KB).  Forms with 194 KB or more (512-token tiles on
+// four slots, 8-bit codes on four slots or at 512 tokens) returned a corrupted tile in
+// some of the calls on the 70B shapes; these never did.
+constexpr int kDx512Slots = 3, kDx512ChunkStages = 4, kDxQ8Slots = 3, kDxQ8ChunkStages = 3;
 
 template <bool kQ8, int kS, int kCS>
 qlora_status launch_dx_variant(dim3 grid, int BN, const CUtensorMap &tmY, const CUtensorMap &tmC,
-                               const CUtensorMap &tmG, const bwdp::Params &p, cudaStream_t st) {
-    const int most = kQ8 ? 256 : (kS == 4 && kCS == 4 ? 256 : 512);   // the largest tile this variant runs
+                               const CUtensorMap &tmG, const CUtensorMap &tmD, const bwdp::Params &p,
+                               cudaStream_t st) {
+    const int most = (kQ8 || kS == 4) ? 256 : 512;   // the largest tile this variant runs
     QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>, bwdp::smem_bytes(most, kQ8, kS, kCS)));
     bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>
-        <<<grid, bwdp::threads_for(kS), bwdp::smem_bytes(BN, kQ8, kS, kCS), st>>>(tmY, tmC, tmG, p);
+        <<<grid, bwdp::threads_for(kS), bwdp::smem_bytes(BN, kQ8, kS, kCS), st>>>(tmY, tmC, tmG, tmD, p);
     return QLORA_OK;
 }
 
@@ -442,7 +449,8 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     CUtensorMap tmY, tmC, tmG;
     QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, box, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
-    const int crow = bwdp::chunk_rows(BN > 256 && !bw.q8 ? kDx512ChunkStages : 4);   // code rows per TMA box
+    // code rows per TMA box
+    const int crow = bwdp::chunk_rows(bw.q8 ? kDxQ8ChunkStages : BN > 256 ? kDx512ChunkStages : 4);
     if (bw.q8)
         QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, crow, 128,
                             CU_TENSOR_MAP_SWIZZLE_128B));
@@ -454,6 +462,13 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
                             CU_TENSOR_MAP_SWIZZLE_128B));
     else
         tmG = tmY;
+    // the dX tile store: [tokens, 128 k] boxes, unswizzled (with splits the epilogue adds into dxacc instead)
+    CUtensorMap tmD;
+    if (!dxacc)
+        QL_TRY(make_tmap_2d(&tmD, dX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, K, std::min(BN, 256),
+                            bwdp::BM, CU_TENSOR_MAP_SWIZZLE_NONE));
+    else
+        tmD = tmY;
     bwdp::Params p;
     p.sc = bw.sc;
     p.d8 = bw.d8;
@@ -475,11 +490,11 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     for (int i = 0; i < 16; ++i) p.level[i] = bw.q8 ? 0.f : bw.level[i];
     dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
     if (bw.q8) {
-        QL_TRY((launch_dx_variant<true, 4, 4>(grid, BN, tmY, tmC, tmG, p, st)));
+        QL_TRY((launch_dx_variant<true, kDxQ8Slots, kDxQ8ChunkStages>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
     } else if (BN > 256) {
-        QL_TRY((launch_dx_variant<false, kDx512Slots, kDx512ChunkStages>(grid, BN, tmY, tmC, tmG, p, st)));
+        QL_TRY((launch_dx_variant<false, kDx512Slots, kDx512ChunkStages>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
     } else {
-        QL_TRY((launch_dx_variant<false, 4, 4>(grid, BN, tmY, tmC, tmG, p, st)));
+        QL_TRY((launch_dx_variant<false, 4, 4>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
     }
     QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
     if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));

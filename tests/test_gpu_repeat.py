@@ -92,3 +92,31 @@ def test_small_m_forward_repeats_bit_exact(N, K, m, flush):
     w, X, dY, A, B, ws = _inputs(N, K, r, 13, M=m)
     out = torch.empty(m, N, dtype=torch.bfloat16, device=DEV)
     _repeat(lambda o: q.qlora_lora_linear_fwd(w, X, A, B, r, 2.0, o, None, ws), out, CALLS_FWD, flush, exact=True)
+
+
+@pytest.mark.parametrize("N,K", [(8192, 8192), (8192, 28672)])
+def test_q8_0_dx_repeats_bit_exact(N, K, flush):
+    """The Q8_0 route's dX, on the same pair-tile kernels, repeats bit for bit as well."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(14)
+    w = q.Q80Weight.empty(N, K)
+    q.qlora_quantize_q8_0(torch.randn(N, K, generator=g, device=DEV) * 0.015, w)
+    dY = torch.randn(M, N, generator=g, device=DEV).to(torch.bfloat16)
+    ws = torch.empty(q.qlora_workspace_bytes(M, N, K, 0), dtype=torch.uint8, device=DEV)
+    out = torch.empty(M, K, dtype=torch.bfloat16, device=DEV)
+    _repeat(lambda o: q.qlora_q8_0_lora_linear_bwd_dx(w, dY, None, None, 0, 0.0, o, None, ws), out, CALLS_DX, flush,
+            exact=True)
+
+
+@pytest.mark.parametrize("N,K", [(8192, 8192), (28672, 8192)])
+def test_q8_0_fwd_repeats_bit_exact(N, K, flush):
+    """The Q8_0 route's forward repeats bit for bit."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(15)
+    w = q.Q80Weight.empty(N, K)
+    q.qlora_quantize_q8_0(torch.randn(N, K, generator=g, device=DEV) * 0.015, w)
+    X = torch.randn(M, K, generator=g, device=DEV).to(torch.bfloat16)
+    ws = torch.empty(q.qlora_workspace_bytes(M, N, K, 0), dtype=torch.uint8, device=DEV)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    _repeat(lambda o: q.qlora_q8_0_lora_linear_fwd(w, X, None, None, 0, 0.0, o, None, ws), out, CALLS_DX, flush,
+            exact=True)
