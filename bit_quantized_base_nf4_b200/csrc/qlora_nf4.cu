@@ -216,10 +216,9 @@ struct DxPlan {
     int64_t pairs, tiles_tok;
     int splits, nb_per_split;
 };
-// Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed (4-bit
-// codes only; see kDx512Slots).  They are taken
+// Tiles of the dX kernel.  wide: 512-token tiles (two accumulators) are allowed.  They are taken
 // when the estimated time of the whole grid is lower: per pair tile about 0.73 us per
-// 64-n stage at 256 tokens and 1.03 us at 512 (measured on the 70B shapes), plus about
+// 64-n stage at 256 tokens and 0.97 us at 512 (measured on the 70B shapes), plus about
 // 10 us of set-up and epilogue, times the number of waves of the pair tiles over the SM pairs.
 DxPlan plan_dx(int64_t M, int64_t N, int64_t K, bool wide) {
     DxPlan d;
@@ -236,7 +235,7 @@ DxPlan plan_dx(int64_t M, int64_t N, int64_t K, bool wide) {
     if (wide && d.splits == 1 && M > 256) {
         const int64_t t512 = ceil_div(M, 512);
         const double w256 = double(ceil_div(tiles, pair_slots)), w512 = double(ceil_div(d.pairs * t512, pair_slots));
-        if (w512 * (double(nb) * 1.03 + 10.0) < w256 * (double(nb) * 0.73 + 10.0)) {
+        if (w512 * (double(nb) * 0.97 + 10.0) < w256 * (double(nb) * 0.73 + 10.0)) {
             d.BN = 512;
             d.tiles_tok = t512;
         }
@@ -420,19 +419,15 @@ qlora_status launch_fwd_pair(const BaseW &bw, const qlora_bf16 *X, int64_t M, in
     return launch_check("fused_fwd_pair_kernel launch");
 }
 
-// dX kernel forms, by shared memory: 4-bit codes take 256-token tiles on four stage
-// slots (= dequant groups) and four-stage code chunks (165 KB), or 512-token tiles on
-// three slots and four-stage chunks (178 KB); 8-bit codes take 256-token tiles on three
-// slots and three-stage chunks (146 KB).  Forms with 194 KB or more (512-token tiles on
-// four slots, 8-bit codes on four slots or at 512 tokens) returned a corrupted tile in
-// some of the calls on the 70B shapes; these never did.
-constexpr int kDx512Slots = 3, kDx512ChunkStages = 4, kDxQ8Slots = 3, kDxQ8ChunkStages = 3;
-
+// dX kernel forms (stage slots = dequant groups kS, stages per code chunk kCS): 4-bit
+// codes take kS = kCS = 4 at every tile (165 KB of shared memory at 256 tokens, 226 KB at
+// 512); 8-bit codes take kS = kCS = 4 up to 256 tokens (198 KB) and kS = kCS = 3 at 512
+// (194 KB: four-stage 8-bit chunks do not fit beside the 512-token rings).
 template <bool kQ8, int kS, int kCS>
-qlora_status launch_dx_variant(dim3 grid, int BN, const CUtensorMap &tmY, const CUtensorMap &tmC,
+qlora_status launch_dx_variant(dim3 grid, int BN, int most, const CUtensorMap &tmY, const CUtensorMap &tmC,
                                const CUtensorMap &tmG, const CUtensorMap &tmD, const bwdp::Params &p,
                                cudaStream_t st) {
-    const int most = (kQ8 || kS == 4) ? 256 : 512;   // the largest tile this variant runs
+    // most: the largest tile this form runs, which sets its shared-memory limit
     QL_TRY(set_smem(bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>, bwdp::smem_bytes(most, kQ8, kS, kCS)));
     bwdp::fused_bwd_pair_kernel<kQ8, kS, kCS>
         <<<grid, bwdp::threads_for(kS), bwdp::smem_bytes(BN, kQ8, kS, kCS), st>>>(tmY, tmC, tmG, tmD, p);
@@ -449,8 +444,7 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     CUtensorMap tmY, tmC, tmG;
     QL_TRY(make_tmap_2d(&tmY, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, box, 64,
                         CU_TENSOR_MAP_SWIZZLE_128B));
-    // code rows per TMA box
-    const int crow = bwdp::chunk_rows(bw.q8 ? kDxQ8ChunkStages : BN > 256 ? kDx512ChunkStages : 4);
+    const int crow = bwdp::chunk_rows(bw.q8 && BN > 256 ? 3 : 4);   // code rows per TMA box
     if (bw.q8)
         QL_TRY(make_tmap_2d(&tmC, bw.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, crow, 128,
                             CU_TENSOR_MAP_SWIZZLE_128B));
@@ -489,13 +483,12 @@ qlora_status launch_dx_pair(const BaseW &bw, const DxPlan &g, const qlora_bf16 *
     p.raster_group = ras.group;
     for (int i = 0; i < 16; ++i) p.level[i] = bw.q8 ? 0.f : bw.level[i];
     dim3 grid(static_cast<unsigned>(2 * g.pairs), static_cast<unsigned>(g.tiles_tok), static_cast<unsigned>(g.splits));
-    if (bw.q8) {
-        QL_TRY((launch_dx_variant<true, kDxQ8Slots, kDxQ8ChunkStages>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
-    } else if (BN > 256) {
-        QL_TRY((launch_dx_variant<false, kDx512Slots, kDx512ChunkStages>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
-    } else {
-        QL_TRY((launch_dx_variant<false, 4, 4>(grid, BN, tmY, tmC, tmG, tmD, p, st)));
-    }
+    if (bw.q8 && BN > 256)
+        QL_TRY((launch_dx_variant<true, 3, 3>(grid, BN, 512, tmY, tmC, tmG, tmD, p, st)));
+    else if (bw.q8)
+        QL_TRY((launch_dx_variant<true, 4, 4>(grid, BN, 256, tmY, tmC, tmG, tmD, p, st)));
+    else
+        QL_TRY((launch_dx_variant<false, 4, 4>(grid, BN, 512, tmY, tmC, tmG, tmD, p, st)));
     QL_TRY(launch_check("fused_bwd_pair_kernel launch"));
     if (dxacc) QL_TRY(launch_finalize(dxacc, M * K, 1.0f, dX, nullptr, st));
     return QLORA_OK;
@@ -915,7 +908,7 @@ qlora_status qlora_q8_0_lora_linear_bwd_dx(const qlora_q8_0_weight *w, const qlo
     QL_TRY(check_rank(r, scaling, A, B));
     const int64_t N = w->n_out, K = w->n_in;
     if (N % 8) return fail(QLORA_ERR_SHAPE, "n_out (%lld) must be a multiple of 8 for the dX pass", (long long)N);
-    const DxPlan g = plan_dx(M, N, K, false);
+    const DxPlan g = plan_dx(M, N, K, true);
     const bool split = g.splits > 1;
     const WsLayout L = ws_layout(M, K, r, split);
     QL_TRY(check_ws(ws, ws_bytes, L.total));
