@@ -40,10 +40,10 @@ CSRC = os.path.join(ROOT, "bit_quantized_base_nf4_b200", "csrc")
 # hash of the kernel sources that capture ran; a source change makes the figure stale
 # and the bench then reports null
 KERNEL_TRAFFIC = {
-    # attention 170.1 + 47.1 MB, FFN up 852.0 + 58.8 MB, FFN down 893.5 + 212.0 MB
-    "dx": {"bytes": 2233458944, "src_sha": "5645f127b9703739"},
-    # attention 117.7 + 51.8 MB, FFN up 1951.7 + 221.4 MB, FFN down 1169.7 + 58.5 MB
-    "fwd": {"bytes": 3570799616, "src_sha": "5c58c99a5d9be592"},
+    # attention 161.1 + 46.1 MB, FFN up 852.4 + 58.6 MB, FFN down 882.2 + 211.5 MB
+    "dx": {"bytes": 2211865600, "src_sha": "98464bdd14b3ae12"},
+    # attention 126.7 + 49.9 MB, FFN up 1873.5 + 222.7 MB, FFN down 1169.6 + 58.3 MB
+    "fwd": {"bytes": 3500716800, "src_sha": "195e2e8f20122b26"},
 }
 
 
