@@ -301,8 +301,8 @@ qlora_status launch_skinny(const void *P, int p_mn, const void *Q, int q_mn, int
     p.ld_j = ld_j;
     const int smem = smem_bytes(p.stages, p.q_bytes);
     QL_TRY(set_smem(skinny_mma_kernel, smem));
-    // stream-K: one CTA per SM, each a contiguous run of (tile, stage) units
-    const int64_t grid = std::min<int64_t>(p.units, sm_count());
+    // stream-K: two CTAs per SM, each a contiguous run of (tile, stage) units
+    const int64_t grid = std::min<int64_t>(p.units, 2 * sm_count());
     skinny_mma_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tmP, tmQ, p);
     return launch_check("skinny_mma_kernel launch");
 }
