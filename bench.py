@@ -40,10 +40,10 @@ CSRC = os.path.join(ROOT, "bit_quantized_base_nf4_b200", "csrc")
 # hash of the kernel sources that capture ran; a source change makes the figure stale
 # and the bench then reports null
 KERNEL_TRAFFIC = {
-    # attention 161.1 + 46.1 MB, FFN up 852.4 + 58.6 MB, FFN down 882.2 + 211.5 MB
-    "dx": {"bytes": 2211865600, "src_sha": "98464bdd14b3ae12"},
-    # attention 126.7 + 49.9 MB, FFN up 1873.5 + 222.7 MB, FFN down 1169.6 + 58.3 MB
-    "fwd": {"bytes": 3500716800, "src_sha": "195e2e8f20122b26"},
+    # attention 162.1 + 46.2 MB, FFN up 852.0 + 57.9 MB, FFN down 847.1 + 211.6 MB
+    "dx": {"bytes": 2176886272, "src_sha": "8d831963ce15634a"},
+    # attention 111.4 + 51.2 MB, FFN up 1952.1 + 222.3 MB, FFN down 1168.5 + 58.7 MB
+    "fwd": {"bytes": 3564198400, "src_sha": "08e3f1cc905141cf"},
 }
 
 
