@@ -760,6 +760,8 @@ NCU_CASES = {
     # name: (list of (N, K), M, r, call run per matrix and step)
     "decode_m1": ([(4096, 4096)], 1, 8, "fwd"),
     "decode_m16": ([(4096, 4096)], 16, 8, "fwd"),
+    # the 7B down projection at M = 1 (11 stages of 1024 k per unit: the steady state)
+    "decode_m1_down": ([(4096, 11008)], 1, 0, "fwd"),
     "dx_70b_attn": ([(8192, 8192)], 4096, 0, "dx"),
     "fwd_70b_attn": ([(8192, 8192)], 4096, 0, "fwd"),
     # the forward with the adapter: the rank-r product U = X A^T, then the GEMM

@@ -5,9 +5,11 @@
 // With at most 16 tokens the forward is bound by streaming the packed weight
 // (0.516 B per weight) from HBM.  tcgen05 cannot keep up at such a narrow N (its
 // per-instruction cost is paid for 128 x 16 x 16 of work), so the contraction runs
-// on warp MMAs, mma.sync m16n8k16 bf16 -> fp32, with the tokens as the m16 operand
-// (rows past M are zero) and eight dequantized W rows as the n8 operand, built in
-// registers from codes through a byte -> bf16x2 table.
+// on warp MMAs, mma.sync m16n8k16 bf16 -> fp32, with sixteen W rows as the m16
+// operand and the tokens as the n8 operand (one or two 8-token tiles; columns past M
+// are zero).  The W operand is W' = bf16(level * bf16(s'_b)), the same values the
+// tensor-core kernels use, built in registers from the codes through a byte -> bf16x2
+// table and one bf16x2 multiply per two weights.
 //
 // Work split.  A unit is 32 W rows over all of K, so no partial sum ever leaves its
 // CTA.  One persistent CTA per SM takes a contiguous run of units.
@@ -23,21 +25,22 @@
 //   - block scales of a unit: one bulk copy of its 32 x K/64 bytes (contiguous in the
 //     packed layout) plus the unit's second-level steps, double-buffered per unit.
 //
-// Fragment mapping.  Consumer warp w takes block pairs w % 4 and w % 4 + 4 of each
-// stage and n8 groups 2(w/4), 2(w/4)+1 of the unit.  For a block pair P, lane (g, t)
-// owns 32 consecutive weights: half t % 2 of block 2P + t/2, i.e. one 16-byte unit of
-// the swizzled code row, which it reads with one conflict-free 128-bit load.  MMA
-// column g is W row sigma(g) = 4 (g % 2) + g / 2 of the n8 group, chosen so that
-// the two rows read by each quarter-warp fall in different swizzle halves.  In
-// k-step j the lane supplies weights 4j .. 4j+3 of its 32 as B and the activations
-// at the same k positions as A; the MMA sums over its k slots in any order, so this
-// pairing only has to agree between A and B.  Each group keeps two accumulators (even
-// and odd k-steps) and the two groups alternate, so four independent MMA chains are
-// in flight per warp.
+// Fragment mapping.  Consumer warp w takes rows 16 (w % 2) .. +15 of the unit and the
+// four blocks of 256-k chunk w / 2 of each stage.  In a block, lane (g, t) owns rows g
+// and g + 8 of its tile and the 16 weights k = 16t .. 16t + 15 of each: 8 code bytes
+// per row, one 64-bit load from the swizzled code row.  k-step q takes bytes 2q and
+// 2q + 1 (k = 16t + 4q + {0,1} in slots 2t, 2t+1 and k = 16t + 4q + {2,3} in slots
+// 2t+8, 2t+9); the lane's activations of token g (and g + 8) at the same 16 k are two
+// 128-bit loads.  The MMA sums over its k slots in any order, so this pairing only has
+// to agree between the two operands.  A table lookup is one byte permute and one
+// 32-bit shared load per two weights.  A stage's four blocks are straight-line code
+// (no per-block branch) into four (two for 16 tokens) accumulator sets, so their MMA
+// chains overlap.
 //
-// The adapter product U = X A^T uses the same loop with the rows of A as extra n8
-// operands; every CTA computes it during its first unit and keeps it in shared
-// memory for the adapter term of all its units.
+// The adapter product U = X A^T uses the same loop with the rows of A (bf16, r <= 16)
+// as a second m16 operand; the warps of the first row tile compute it during the
+// CTA's first unit, and the CTA keeps it in shared memory for the adapter term of all
+// its units.
 //
 // Overlap with the preceding kernel (programmatic dependent launch): before waiting
 // on the preceding grid a CTA only builds its table and initialises its barriers;
@@ -45,6 +48,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -65,7 +69,7 @@ constexpr int kCodeStage = kRows * kStageK / 2; // 16 KB
 constexpr int kLutBytes = 256 * 32 * 4;         // one bf16x2 per byte value per lane
 constexpr int kMaxCodeStages = 6;
 constexpr int kMaxXaStages = 4;
-constexpr int kPartFloats = 4 * kRows * 16;     // [block pair][row][token]
+constexpr int kPartFloats = 4 * kRows * 16;     // [chunk][row][token]
 constexpr int kSmemLimit = 232448;
 
 struct Params {
@@ -85,13 +89,22 @@ struct Params {
     float level[16];
 };
 
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+// d += A B
+__device__ __forceinline__ void mma_acc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                        uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// This lane's table entry for byte c of w: (level[lo], level[hi]) as bf16x2.  The
+// table is written before the CTA's first __syncthreads and only read afterwards, and
+// w comes from a barrier-guarded load, so the load is free to move with its address.
+__device__ __forceinline__ uint32_t lut_at(uint32_t lut_lane, uint32_t w, int c) {
+    const uint32_t e = __byte_perm(w, 0u, 0x4440u | static_cast<uint32_t>(c));
+    uint32_t v;
+    asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(lut_lane + (e << 7)));
+    return v;
 }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -269,33 +282,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------------- consumers
     // A wait that times out sets the CTA's abort flag and the device error word (which
     // the host reports); the consumers then run on without waiting, so that all eight
-    // warps still reach every named barrier and the CTA exits.
-    const int pr = warp & 3, gs = warp >> 2;
+    // consumer warps still reach every named barrier and the CTA exits.
+    const int rt = warp & 1, bq = warp >> 1;            // row tile (16 rows), 256-k chunk of each stage
     const int g = lane >> 2, t = lane & 3;
-    const int sg = ((g & 1) << 2) | (g >> 1);          // W row (in its n8 group) of MMA column g
     const int ctid = threadIdx.x;                      // 0 .. kConsumers-1
-    const uint32_t lut = smem_u32(smem) + lane * 4;
+    const uint32_t lut_lane = smem_u32(smem) + lane * 4;
     const uint32_t code_base = smem_u32(smem + p.off_code);
     const uint32_t xa_base = smem_u32(smem + p.off_xa);
     float *part = reinterpret_cast<float *>(smem + p.off_part);
     float *upart = reinterpret_cast<float *>(smem + p.off_upart);
     float *ufin = reinterpret_cast<float *>(smem + p.off_ufin);
     const bool tok0 = g < p.M, tok1 = NT > 1 && g + 8 < p.M;
-    const bool do_u = gs < nA;
+    const bool do_u = rt == 0 && p.r > 0;               // these warps also form U = X A^T
+    const bool arow1 = g + 8 < p.r;                     // A row g + 8 exists (r = 16)
     const int brow = ctid & 31;                         // epilogue row
-    const uint32_t u4 = 4 * (t & 1);                    // first 16-byte unit of this lane's half block
-    // per block pair h (pairs pr and pr + 4): the 64-k chunk this lane reads, its X lines
-    // (line = chunk * M + token; the swizzle XORs the unit with line % 8) and its code unit
-    int chunk[2];
-    uint32_t xl0[2], xl1[2], c_off[2], a_off[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        chunk[h] = 2 * (pr + 4 * h) + (t >> 1);
-        xl0[h] = uint32_t(chunk[h] * p.M + g);
-        xl1[h] = uint32_t(chunk[h] * p.M + g + 8);
-        c_off[h] = uint32_t(((pr >> 1) + 2 * h) * (kRows * 128) + (((4 * (pr & 1) + t) ^ sg) << 4));
-        a_off[h] = uint32_t(p.M * (kStageBlocks * 128) + (chunk[h] * p.r + 8 * gs + g) * 128);
-    }
+    const int R0 = 16 * rt + g;                         // unit rows of this lane: R0 and R0 + 8
+    // this lane's 8 code bytes of block c of its chunk in row R0: 16-byte unit 2c + t/2
+    // of the row's 128 bytes (stored at unit (2c + t/2) ^ (R0 % 8), R0 % 8 = g), half t%2
+    const uint32_t c_lane =
+        code_base + uint32_t(bq * (kRows * 128) + R0 * 128 + ((((t >> 1) ^ g) << 4) | ((t & 1) << 3)));
+    // X and A lines of the stage's 64-k chunks: line * 128 + (unit ^ (line % 8)) * 16
+    auto line_addr = [](uint32_t base, int line, int unit) {
+        return base + uint32_t(line) * 128u + (uint32_t(unit ^ (line & 7)) << 4);
+    };
 
     int cslot = 0, cph = 0, xslot = 0, xph = 0;
     for (int ui = 0; ui < nu; ++ui) {
@@ -317,85 +326,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         // flat block index of the unit's first block, modulo one second-level group: the
         // unit's steps were copied starting from the group holding that block
         const int fb_lo = static_cast<int>((int64_t(n0) * KB) & 255);
-        // per group: this lane's W row in the code box and in the unit's scale rows
-        uint32_t row_off[2];
-        int row_q[2];
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int row = 8 * (2 * gs + gg) + sg;
-            row_off[gg] = uint32_t(row * 128);
-            row_q[gg] = row * KB;
-        }
+        const int row_q0 = R0 * KB, row_q1 = (R0 + 8) * KB;
 
-        float acc[2][2][4], accU[2][4];
+        // the block's scale s'_b = q_b * d_g of a row, rounded to bf16 and paired; a block
+        // past the end of K gets 0 (its codes and activations are the copies' zero fill)
+        auto scale_pair = [&](int row_q, int kb) {
+            const float sv = static_cast<float>(lds_u8(sq + uint32_t(row_q + kb))) *
+                             lds_f32(s2 + uint32_t(((fb_lo + row_q + kb) >> 8) << 2));
+            __nv_bfloat162 v = __float2bfloat162_rn(kb < KB ? sv : 0.f);
+            return *reinterpret_cast<uint32_t *>(&v);
+        };
+        // kAcc accumulator sets, one per block modulo kAcc, keep independent MMA chains
+        constexpr int kAcc = NT == 1 ? 4 : 2;
+        float acc[kAcc][NT][4], accU[NT][4];
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+        for (int a = 0; a < NT; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) acc[0][a][b] = acc[1][a][b] = accU[a][b] = 0.f;
+            for (int b = 0; b < 4; ++b) {
+                accU[a][b] = 0.f;
+#pragma unroll
+                for (int h = 0; h < kAcc; ++h) acc[h][a][b] = 0.f;
+            }
+        // one stage of this warp: the four blocks of its chunk, straight-line code
+        auto stage = [&](auto with_u, uint32_t cs, uint32_t xs, int j) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int kc = 4 * bq + c;                   // 64-k chunk of the stage
+                const int kb = j * kStageBlocks + kc;        // block of the row
+                // rows R0, R0 + 8: 16 weights each, k = 16t .. 16t + 15 of the block
+                const uint32_t ca = cs ^ uint32_t(c << 5);
+                const uint2 w0 = lds64(ca);
+                const uint2 w1 = lds64(ca + 8 * 128);
+                // tokens g and g + 8 at the same 16 k
+                uint4 xa0 = make_uint4(0, 0, 0, 0), xb0 = xa0, xa1 = xa0, xb1 = xa0;
+                if (tok0) {
+                    xa0 = lds128(line_addr(xs, kc * p.M + g, 2 * t));
+                    xb0 = lds128(line_addr(xs, kc * p.M + g, 2 * t + 1));
+                }
+                if (tok1) {
+                    xa1 = lds128(line_addr(xs, kc * p.M + g + 8, 2 * t));
+                    xb1 = lds128(line_addr(xs, kc * p.M + g + 8, 2 * t + 1));
+                }
+                const uint32_t s0 = scale_pair(row_q0, kb), s1 = scale_pair(row_q1, kb);
+                // k-step q takes bytes 2q, 2q+1 of each row's 8: k = 16t + 4q + {0,1} in
+                // slots 2t, 2t+1 and 16t + 4q + {2,3} in slots 2t+8, 2t+9; the activations
+                // supply the same k in the same slots.  W' = bf16(level * bf16(s'_b)).
+                const uint32_t xw0[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xb0.x, xb0.y, xb0.z, xb0.w};
+                const uint32_t xw1[8] = {xa1.x, xa1.y, xa1.z, xa1.w, xb1.x, xb1.y, xb1.z, xb1.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t r0w = (q < 2) ? w0.x : w0.y, r1w = (q < 2) ? w1.x : w1.y;
+                    const int by = 2 * (q & 1);
+                    const uint32_t a0 = bf16x2_mul(lut_at(lut_lane, r0w, by), s0);
+                    const uint32_t a2 = bf16x2_mul(lut_at(lut_lane, r0w, by + 1), s0);
+                    const uint32_t a1 = bf16x2_mul(lut_at(lut_lane, r1w, by), s1);
+                    const uint32_t a3 = bf16x2_mul(lut_at(lut_lane, r1w, by + 1), s1);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const uint32_t *xw = nt ? xw1 : xw0;
+                        mma_acc(acc[c % kAcc][nt], a0, a1, a2, a3, xw[2 * q], xw[2 * q + 1]);
+                    }
+                }
+                if constexpr (decltype(with_u)::value) {
+                    // A rows g and g + 8 at the same 16 k, straight from the stage (bf16)
+                    const int al = kc * p.r + g;
+                    const uint32_t ab = xs + uint32_t(p.M * (kStageBlocks * 128));
+                    const uint4 aa0 = lds128(line_addr(ab, al, 2 * t)), ab0 = lds128(line_addr(ab, al, 2 * t + 1));
+                    uint4 aa1 = make_uint4(0, 0, 0, 0), ab1 = aa1;
+                    if (arow1) {
+                        aa1 = lds128(line_addr(ab, al + 8, 2 * t));
+                        ab1 = lds128(line_addr(ab, al + 8, 2 * t + 1));
+                    }
+                    const uint32_t aw0[8] = {aa0.x, aa0.y, aa0.z, aa0.w, ab0.x, ab0.y, ab0.z, ab0.w};
+                    const uint32_t aw1[8] = {aa1.x, aa1.y, aa1.z, aa1.w, ab1.x, ab1.y, ab1.z, ab1.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t *xw = nt ? xw1 : xw0;
+                            mma_acc(accU[nt], aw0[2 * q], aw1[2 * q], aw0[2 * q + 1], aw1[2 * q + 1], xw[2 * q],
+                                    xw[2 * q + 1]);
+                        }
+                }
+            }
+        };
+        const bool u_here = first && do_u;
         for (int j = 0; j < nst; ++j) {
             if (lane == 0) {   // one lane polls; the warp barrier orders the others after it
                 mbar_wait(&code_full[cslot], cph, abort_flag);
                 mbar_wait(&xa_full[xslot], xph, abort_flag);
             }
             __syncwarp();
-            const uint32_t cs = code_base + uint32_t(cslot * kCodeStage);
+            const uint32_t cs = c_lane + uint32_t(cslot * kCodeStage);
             const uint32_t xs = xa_base + uint32_t(xslot * p.xa_stage);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int kb = j * kStageBlocks + chunk[h];
-                const bool kv = kb < KB;
-                uint4 xw[4], xh[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    xw[q] = tok0 ? lds128(xs + xl0[h] * 128 + (((u4 + q) ^ (xl0[h] & 7)) << 4)) : make_uint4(0, 0, 0, 0);
-                    xh[q] = tok1 ? lds128(xs + xl1[h] * 128 + (((u4 + q) ^ (xl1[h] & 7)) << 4)) : make_uint4(0, 0, 0, 0);
-                }
-                uint32_t sc[2];
-                uint4 cw[2];
-#pragma unroll
-                for (int gg = 0; gg < 2; ++gg) {
-                    sc[gg] = 0;
-                    if (kv) {
-                        const uint32_t q = lds_u8(sq + uint32_t(row_q[gg] + kb));
-                        const float d = lds_f32(s2 + uint32_t(((fb_lo + row_q[gg] + kb) >> 8) << 2));
-                        __nv_bfloat162 s2b = __float2bfloat162_rn(__fmul_rn(static_cast<float>(q), d));
-                        sc[gg] = *reinterpret_cast<uint32_t *>(&s2b);
-                    }
-                    cw[gg] = lds128(cs + c_off[h] + row_off[gg]);
-                }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const uint4 &xa = xw[jj >> 1];
-                    const uint4 &xb = xh[jj >> 1];
-                    const uint32_t a0 = (jj & 1) ? xa.z : xa.x, a2 = (jj & 1) ? xa.w : xa.y;
-                    const uint32_t a1 = (jj & 1) ? xb.z : xb.x, a3 = (jj & 1) ? xb.w : xb.y;
-#pragma unroll
-                    for (int gg = 0; gg < 2; ++gg) {
-                        const uint32_t cwv[4] = {cw[gg].x, cw[gg].y, cw[gg].z, cw[gg].w};
-                        const uint32_t word = cwv[jj >> 1];
-                        const uint32_t sh = 16 * (jj & 1);
-                        const uint32_t e0 = (word >> sh) & 0xFFu, e1 = (word >> (sh + 8)) & 0xFFu;
-                        const uint32_t b0 = bf16x2_mul(lds32_const(lut + (e0 << 7)), sc[gg]);
-                        const uint32_t b1 = bf16x2_mul(lds32_const(lut + (e1 << 7)), sc[gg]);
-                        mma_bf16_16816(acc[gg][jj & 1], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, b0, b1);
-                    }
-                }
-                if (first && do_u) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 aw = lds128(xs + a_off[h] + (((u4 + q) ^ g) << 4));
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint4 &xa = xw[q];
-                            const uint4 &xb = xh[q];
-                            const uint32_t a0 = hh ? xa.z : xa.x, a2 = hh ? xa.w : xa.y;
-                            const uint32_t a1 = hh ? xb.z : xb.x, a3 = hh ? xb.w : xb.y;
-                            mma_bf16_16816(accU[hh], a0, NT > 1 ? a1 : 0u, a2, NT > 1 ? a3 : 0u, hh ? aw.z : aw.x,
-                                           hh ? aw.w : aw.y);
-                        }
-                    }
-                }
-            }
+            if (u_here) stage(std::true_type{}, cs, xs, j);
+            else stage(std::false_type{}, cs, xs, j);
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&code_empty[cslot]);
@@ -404,34 +429,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++cslot == p.dc) { cslot = 0; cph ^= 1; }
             if (++xslot == p.dx) { xslot = 0; xph ^= 1; }
         }
+#pragma unroll
+        for (int h = 1; h < kAcc; ++h)
+#pragma unroll
+            for (int a = 0; a < NT; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[0][a][b] += acc[h][a][b];
         __syncwarp();
         if (lane == 0) mbar_arrive(&sc_empty[sb]);
 
-        // partial sums of block pairs pr, pr + 4 -> part[pr][row][token]
-        float *pb = part + pr * kRows * 16;
+        // partial sums of chunk bq -> part[bq][row][token]; D[row][token] of the MMA has
+        // rows g, g + 8 and tokens 2t, 2t + 1 of each 8-token tile in this lane
+        float *pb = part + bq * kRows * 16;
 #pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int grp = 2 * gs + gg;
-            const int c0 = 2 * t, c1 = 2 * t + 1;
-            const int R0 = 8 * grp + (((c0 & 1) << 2) | (c0 >> 1));
-            const int R1 = 8 * grp + (((c1 & 1) << 2) | (c1 >> 1));
-            pb[R0 * 16 + g] = acc[gg][0][0] + acc[gg][1][0];
-            pb[R1 * 16 + g] = acc[gg][0][1] + acc[gg][1][1];
-            pb[R0 * 16 + g + 8] = acc[gg][0][2] + acc[gg][1][2];
-            pb[R1 * 16 + g + 8] = acc[gg][0][3] + acc[gg][1][3];
+        for (int nt = 0; nt < NT; ++nt) {
+            const int m0 = 8 * nt + 2 * t;
+            pb[R0 * 16 + m0] = acc[0][nt][0];
+            pb[R0 * 16 + m0 + 1] = acc[0][nt][1];
+            pb[(R0 + 8) * 16 + m0] = acc[0][nt][2];
+            pb[(R0 + 8) * 16 + m0 + 1] = acc[0][nt][3];
         }
         if (first && do_u) {
-            float *ub = upart + pr * 256;
-            const int j0 = 8 * gs + 2 * t;
-            ub[g * 16 + j0] = accU[0][0] + accU[1][0];
-            ub[g * 16 + j0 + 1] = accU[0][1] + accU[1][1];
-            ub[(g + 8) * 16 + j0] = accU[0][2] + accU[1][2];
-            ub[(g + 8) * 16 + j0 + 1] = accU[0][3] + accU[1][3];
+            float *ub = upart + bq * 256;   // [adapter row][token]
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m0 = 8 * nt + 2 * t;
+                ub[g * 16 + m0] = accU[nt][0];
+                ub[g * 16 + m0 + 1] = accU[nt][1];
+                ub[(g + 8) * 16 + m0] = accU[nt][2];
+                ub[(g + 8) * 16 + m0 + 1] = accU[nt][3];
+            }
         }
         consumer_sync();
         if (first && p.r > 0) {
-            for (int e = ctid; e < 256; e += kConsumers)
-                ufin[e] = upart[e] + upart[256 + e] + upart[512 + e] + upart[768 + e];
+            // ufin[token][adapter row]
+            for (int e = ctid; e < 256; e += kConsumers) {
+                const int m = e >> 4, jr = e & 15;
+                const int src = jr * 16 + m;
+                ufin[e] = upart[src] + upart[256 + src] + upart[512 + src] + upart[768 + src];
+            }
             consumer_sync();
             if (p.U_save && blockIdx.x == 0) {
                 for (int e = ctid; e < p.M * p.r; e += kConsumers) {
